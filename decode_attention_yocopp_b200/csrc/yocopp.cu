@@ -1,0 +1,349 @@
+// yocopp C ABI: host-side argument checks, TMA descriptor encoding, split
+// planning and kernel launches for the YOCO++ compose/append and the shared-
+// cache decode attention.  One translation unit holds every kernel so the
+// device status word is a single symbol.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "compose_append.cuh"
+#include "decode_attn.cuh"
+
+namespace yocopp {
+namespace {
+
+constexpr int kMaxBatch = 8192;
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
+
+int g_test_drop_tile = -1;
+uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int elem_bytes(int dtype) { return dtype == YOCOPP_BF16 ? 2 : (dtype == YOCOPP_F32 ? 4 : 0); }
+
+int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
+int sm_count(int dev) {
+    static int cache[kMaxDevices] = {0};
+    if (dev < 0 || dev >= kMaxDevices) return -1;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return -1;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+    static EncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeFn>(p);
+    });
+    return fn;
+}
+
+// 2-D view of a cache tensor: rows of head_dim elements; 128-byte swizzled
+// boxes of (128 / elem) x box_rows.
+bool encode_rows(CUtensorMap* map, void* base, int dtype, int head_dim, int64_t rows, int box_rows) {
+    EncodeFn fn = encode_fn();
+    if (!fn) return false;
+    const int eb = elem_bytes(dtype);
+    cuuint64_t gdim[2] = {cuuint64_t(head_dim), cuuint64_t(rows)};
+    cuuint64_t gstride[1] = {cuuint64_t(head_dim) * eb};
+    cuuint32_t box[2] = {cuuint32_t(128 / eb), cuuint32_t(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, dtype == YOCOPP_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+              base, gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Shape checks shared by both entry points; returns YOCOPP_OK or an error.
+int32_t check_cache(const yocopp_cache* c) {
+    if (c == nullptr || c->k == nullptr || c->v == nullptr) return YOCOPP_EINVAL;
+    if (elem_bytes(c->dtype) == 0) return YOCOPP_EDTYPE;
+    if (c->head_dim != 64 && c->head_dim != 128) return YOCOPP_EINVAL;
+    if (c->batch < 1 || c->batch > kMaxBatch || c->num_kv_heads < 1 || c->capacity < 1) return YOCOPP_EINVAL;
+    if (!aligned(c->k, 16) || !aligned(c->v, 16)) return YOCOPP_EINVAL;
+    int64_t rows;
+    if (c->block_table != nullptr) {
+        const int bs = c->block_size;
+        if (bs != 16 && bs != 32 && bs != 64 && bs != 128 && bs != 256) return YOCOPP_EINVAL;
+        if (c->max_blocks_per_seq < 1 || c->num_blocks < 1) return YOCOPP_EINVAL;
+        if (int64_t(bs) * c->max_blocks_per_seq != c->capacity) return YOCOPP_EINVAL;
+        rows = int64_t(c->num_blocks) * c->num_kv_heads * bs;
+    } else {
+        rows = int64_t(c->batch) * c->num_kv_heads * c->capacity;
+    }
+    if (rows >= (int64_t(1) << 31)) return YOCOPP_EINVAL;  // 32-bit row coordinates
+    return YOCOPP_OK;
+}
+
+int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? YOCOPP_OK : YOCOPP_ECUDA; }
+
+// ---------------------------------------------------------------- compose
+template <typename T, int ROWB>
+int32_t launch_compose(ComposeParams& p, cudaStream_t st) {
+    const int dev = current_device();
+    const int sms = sm_count(dev);
+    if (sms <= 0) return YOCOPP_ECUDA;
+    const int64_t nchunks = p.total_rows * (ROWB / 16);
+    int64_t grid = (nchunks + 511) / 512;
+    if (grid > int64_t(sms) * 8) grid = int64_t(sms) * 8;
+    if (grid < 1) grid = 1;
+    const size_t smem = p.cu_new ? size_t(p.batch + 1) * sizeof(int) : 0;
+    compose_append_kernel<T, ROWB><<<unsigned(grid), 256, smem, st>>>(p);
+    return cuda_status(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------- decode
+struct DecodeLaunch {
+    int w, stages, tile;
+};
+
+template <typename T, int D>
+constexpr DecodeLaunch decode_cfg() {
+    return DecodeLaunch{4, 5, DecodeShape<D, T>::TILE};
+}
+
+template <typename T, int D, int G>
+int32_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, cudaStream_t st) {
+    constexpr DecodeLaunch cfg = decode_cfg<T, D>();
+    constexpr int W = cfg.w, STAGES = cfg.stages;
+    auto kern = decode_split_kernel<T, D, G, W, STAGES>;
+    const size_t smem = DecodeSmem<T, D, G, W, STAGES>::bytes(p.batch);
+    static bool attr_set[kMaxDevices] = {false};
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return YOCOPP_ECUDA;
+    static size_t max_dyn[kMaxDevices] = {0};
+    if (!attr_set[dev]) {
+        int maxopt = 0;
+        cudaFuncAttributes fa;
+        if (cudaDeviceGetAttribute(&maxopt, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+            cudaFuncGetAttributes(&fa, kern) != cudaSuccess)
+            return YOCOPP_ECUDA;
+        max_dyn[dev] = size_t(maxopt) - fa.sharedSizeBytes;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(max_dyn[dev])) != cudaSuccess)
+            return YOCOPP_ECUDA;
+        attr_set[dev] = true;
+    }
+    if (smem > max_dyn[dev]) return YOCOPP_EINVAL;  // batch too large for the shared-memory plan
+    kern<<<p.num_ctas, (W + 1) * 32, smem, st>>>(tk, tv, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return YOCOPP_ECUDA;
+    decode_combine_kernel<T, D, G><<<p.batch * p.hkv, 128, 0, st>>>(p);
+    return cuda_status(cudaGetLastError());
+}
+
+struct WorkspaceLayout {
+    size_t tile_start, m, l, o, total;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WorkspaceLayout workspace_layout(int batch, int hkv, int G, int D, int num_ctas) {
+    const size_t slots = size_t(num_ctas) + size_t(batch) * hkv;
+    WorkspaceLayout w;
+    w.tile_start = 0;
+    w.m = up256(size_t(batch + 1) * sizeof(int));
+    w.l = w.m + up256(slots * G * sizeof(float));
+    w.o = w.l + up256(slots * G * sizeof(float));
+    w.total = w.o + up256(slots * G * D * sizeof(float));
+    return w;
+}
+
+int32_t check_decode_shape(const yocopp_cache* cache, int32_t num_q_heads, int* G) {
+    const int32_t rc = check_cache(cache);
+    if (rc != YOCOPP_OK) return rc;
+    if (num_q_heads < 1 || num_q_heads % cache->num_kv_heads != 0) return YOCOPP_EINVAL;
+    *G = num_q_heads / cache->num_kv_heads;
+    if (*G != 1 && *G != 2 && *G != 4) return YOCOPP_EINVAL;
+    const int tile = (cache->head_dim * elem_bytes(cache->dtype)) <= 256 ? 64 : 32;
+    if (cache->block_table != nullptr && cache->block_size % tile != 0 && tile % cache->block_size != 0)
+        return YOCOPP_EINVAL;
+    const int64_t tiles = int64_t(cache->batch) * cache->num_kv_heads * ((cache->capacity + tile - 1) / tile);
+    if (tiles >= (int64_t(1) << 31)) return YOCOPP_EINVAL;
+    return YOCOPP_OK;
+}
+
+}  // namespace
+}  // namespace yocopp
+
+using namespace yocopp;
+
+extern "C" {
+
+int32_t yocopp_version(void) { return 100; }
+
+const char* yocopp_status_string(int32_t s) {
+    switch (s) {
+        case YOCOPP_OK: return "YOCOPP_OK";
+        case YOCOPP_EINVAL: return "YOCOPP_EINVAL";
+        case YOCOPP_EDTYPE: return "YOCOPP_EDTYPE";
+        case YOCOPP_ECAPACITY: return "YOCOPP_ECAPACITY";
+        case YOCOPP_EWORKSPACE: return "YOCOPP_EWORKSPACE";
+        case YOCOPP_ECUDA: return "YOCOPP_ECUDA";
+        case YOCOPP_EDEVICE_CHECK: return "YOCOPP_EDEVICE_CHECK";
+        case YOCOPP_ETIMEOUT: return "YOCOPP_ETIMEOUT";
+        default: return "YOCOPP_UNKNOWN";
+    }
+}
+
+int32_t yocopp_get_device_status(int32_t reset) {
+    int v = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return YOCOPP_ECUDA;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return YOCOPP_ECUDA;
+    if (reset) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return YOCOPP_ECUDA;
+    }
+    return v;
+}
+
+int32_t yocopp_testing_set_decode_fault(int32_t drop_tile, int64_t wait_limit_ns) {
+    if (wait_limit_ns <= 0) return YOCOPP_EINVAL;
+    g_test_drop_tile = drop_tile < 0 ? -1 : drop_tile;
+    g_wait_limit_ns = uint64_t(wait_limit_ns);
+    return YOCOPP_OK;
+}
+
+int32_t yocopp_compose_append(const void* K1, const void* V1, const void* Ki, const void* Vi,
+                              const float alpha[4], float lambda, const yocopp_cache* cache,
+                              const int32_t* pos, const int32_t* cu_new, int32_t n_uniform,
+                              int64_t total_new, void* stream) {
+    const int32_t rc = check_cache(cache);
+    if (rc != YOCOPP_OK) return rc;
+    if (alpha == nullptr || pos == nullptr || total_new < 0) return YOCOPP_EINVAL;
+    if (!std::isfinite(lambda) || !std::isfinite(alpha[0]) || !std::isfinite(alpha[1]) ||
+        !std::isfinite(alpha[2]) || !std::isfinite(alpha[3]))
+        return YOCOPP_EINVAL;
+    if (cu_new == nullptr) {
+        if (n_uniform < 0 || int64_t(n_uniform) * cache->batch != total_new) return YOCOPP_EINVAL;
+    }
+    if (total_new == 0) return YOCOPP_OK;
+    if (K1 == nullptr || V1 == nullptr || Ki == nullptr || Vi == nullptr) return YOCOPP_EINVAL;
+    if (!aligned(K1, 16) || !aligned(V1, 16) || !aligned(Ki, 16) || !aligned(Vi, 16)) return YOCOPP_EINVAL;
+    if (total_new > (int64_t(1) << 40)) return YOCOPP_EINVAL;
+
+    ComposeParams p;
+    p.k1 = static_cast<const uint8_t*>(K1);
+    p.v1 = static_cast<const uint8_t*>(V1);
+    p.ki = static_cast<const uint8_t*>(Ki);
+    p.vi = static_cast<const uint8_t*>(Vi);
+    p.ck = static_cast<uint8_t*>(cache->k);
+    p.cv = static_cast<uint8_t*>(cache->v);
+    p.block_table = cache->block_table;
+    p.pos = pos;
+    p.cu_new = cu_new;
+    p.ak1 = alpha[0];
+    p.ak2 = alpha[1];
+    p.av1 = alpha[2];
+    p.av2 = alpha[3];
+    p.lam = lambda;
+    p.total_rows = total_new * cache->num_kv_heads;
+    p.hkv = cache->num_kv_heads;
+    p.batch = cache->batch;
+    p.n_uniform = n_uniform;
+    p.capacity = cache->capacity;
+    p.block_size = cache->block_table ? cache->block_size : 0;
+    p.mbps = cache->block_table ? cache->max_blocks_per_seq : 0;
+    p.num_blocks = cache->block_table ? cache->num_blocks : 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int rowb = cache->head_dim * elem_bytes(cache->dtype);
+    if (cache->dtype == YOCOPP_BF16)
+        return rowb == 256 ? launch_compose<__nv_bfloat16, 256>(p, st) : launch_compose<__nv_bfloat16, 128>(p, st);
+    return rowb == 512 ? launch_compose<float, 512>(p, st) : launch_compose<float, 256>(p, st);
+}
+
+int64_t yocopp_decode_attn_workspace_size(const yocopp_cache* cache, int32_t num_q_heads) {
+    int G = 0;
+    const int32_t rc = check_decode_shape(cache, num_q_heads, &G);
+    if (rc != YOCOPP_OK) return rc;
+    const int sms = sm_count(current_device());
+    if (sms <= 0) return YOCOPP_ECUDA;
+    return int64_t(workspace_layout(cache->batch, cache->num_kv_heads, G, cache->head_dim, sms).total);
+}
+
+int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32_t* seq_lens, void* out,
+                           int32_t num_q_heads, float scale, void* workspace, int64_t workspace_bytes,
+                           void* stream) {
+    int G = 0;
+    int32_t rc = check_decode_shape(cache, num_q_heads, &G);
+    if (rc != YOCOPP_OK) return rc;
+    if (q == nullptr || out == nullptr || seq_lens == nullptr) return YOCOPP_EINVAL;
+    if (!aligned(q, 16) || !aligned(out, 16)) return YOCOPP_EINVAL;
+    if (!(scale >= 0.f) || !std::isfinite(scale)) return YOCOPP_EINVAL;
+    const int sms = sm_count(current_device());
+    if (sms <= 0) return YOCOPP_ECUDA;
+    const WorkspaceLayout wl = workspace_layout(cache->batch, cache->num_kv_heads, G, cache->head_dim, sms);
+    if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < int64_t(wl.total))
+        return YOCOPP_EWORKSPACE;
+
+    const int D = cache->head_dim;
+    const int tile = (D * elem_bytes(cache->dtype)) <= 256 ? 64 : 32;
+    const bool paged = cache->block_table != nullptr;
+    const int boxr = paged ? (cache->block_size < tile ? cache->block_size : tile) : tile;
+    const int64_t rows = paged ? int64_t(cache->num_blocks) * cache->num_kv_heads * cache->block_size
+                               : int64_t(cache->batch) * cache->num_kv_heads * cache->capacity;
+    alignas(64) CUtensorMap tk, tv;
+    if (!encode_rows(&tk, cache->k, cache->dtype, D, rows, boxr) ||
+        !encode_rows(&tv, cache->v, cache->dtype, D, rows, boxr))
+        return YOCOPP_ECUDA;
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    DecodeParams p;
+    p.q = static_cast<const uint8_t*>(q);
+    p.out = static_cast<uint8_t*>(out);
+    p.seq_lens = seq_lens;
+    p.block_table = cache->block_table;
+    p.ws_tile_start = reinterpret_cast<int32_t*>(ws + wl.tile_start);
+    p.ws_m = reinterpret_cast<float*>(ws + wl.m);
+    p.ws_l = reinterpret_cast<float*>(ws + wl.l);
+    p.ws_o = reinterpret_cast<float*>(ws + wl.o);
+    const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(float(D));
+    p.qscale = sc * 1.4426950408889634f;
+    p.batch = cache->batch;
+    p.hkv = cache->num_kv_heads;
+    p.hq = num_q_heads;
+    p.capacity = cache->capacity;
+    p.block_size = paged ? cache->block_size : 0;
+    p.mbps = paged ? cache->max_blocks_per_seq : 0;
+    p.num_blocks = paged ? cache->num_blocks : 0;
+    p.boxr = boxr;
+    p.num_ctas = sms;
+    p.drop_tile = g_test_drop_tile;
+    p.wait_limit_ns = g_wait_limit_ns;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+#define YOCOPP_DECODE_CASE(TT, DD)                                             \
+    switch (G) {                                                               \
+        case 1: return launch_decode<TT, DD, 1>(tk, tv, p, st);                \
+        case 2: return launch_decode<TT, DD, 2>(tk, tv, p, st);                \
+        default: return launch_decode<TT, DD, 4>(tk, tv, p, st);               \
+    }
+    if (cache->dtype == YOCOPP_BF16) {
+        if (D == 128) { YOCOPP_DECODE_CASE(__nv_bfloat16, 128) }
+        YOCOPP_DECODE_CASE(__nv_bfloat16, 64)
+    }
+    if (D == 128) { YOCOPP_DECODE_CASE(float, 128) }
+    YOCOPP_DECODE_CASE(float, 64)
+#undef YOCOPP_DECODE_CASE
+}
+
+}  // extern "C"

@@ -339,25 +339,32 @@ class Workload:
         return 2 * sum(self.lens) * self.hkv * self.d * self.elem_bytes
 
 
+def _f32(x: float) -> float:
+    """The residual weights are fp32 parameters (and cross the C ABI as fp32), so
+    every workload's alpha is an exactly fp32-representable value that both the
+    kernels and the oracle receive unchanged."""
+    return float(np.float32(x))
+
+
 def _alpha_offsets(seed: int, layers: int) -> Dict[int, Tuple[float, float, float, float]]:
     """alpha ~ U(-0.05, 0.05) offset from the stated init (0, 1/lambda), 4 draws per layer."""
     out = {}
     for i in range(2, layers // 2 + 1):
         u = uniform01(seed, _SCALARS, 4, offset=16 * i) * 0.1 - 0.05
-        out[i] = (float(u[0]), 1.0 / LAMBDA_DEFAULT + float(u[1]),
-                  float(u[2]), 1.0 / LAMBDA_DEFAULT + float(u[3]))
+        out[i] = (_f32(u[0]), _f32(1.0 / LAMBDA_DEFAULT + float(u[1])),
+                  _f32(u[2]), _f32(1.0 / LAMBDA_DEFAULT + float(u[3])))
     return out
 
 
 def _alpha_init(layers: int, lam: float = LAMBDA_DEFAULT) -> Dict[int, Tuple[float, float, float, float]]:
-    return {i: (0.0, 1.0 / lam, 0.0, 1.0 / lam) for i in range(2, layers // 2 + 1)}
+    return {i: (0.0, _f32(1.0 / lam), 0.0, _f32(1.0 / lam)) for i in range(2, layers // 2 + 1)}
 
 
 def config(n: int, planted_mode: str = "aligned", **over) -> Workload:
     """The five workloads. ``over`` replaces fields (e.g. smaller lens for tests)."""
     seed = 20261202 + 1000 * n
     if n == 1:
-        a = (0.1, 1.0 / 35 + 0.01)
+        a = (_f32(0.1), _f32(1.0 / 35 + 0.01))
         w = Workload("tiny", 1, 4, 1, 1, 1, 64, "f32", [256], alpha={2: (a[0], a[1], a[0], a[1])}, seed=seed)
     elif n == 2:
         w = Workload("b4_t4096", 2, 24, 4, 32, 8, 128, "bf16", [4096] * 4, alpha=_alpha_offsets(seed, 24), seed=seed)

@@ -1,0 +1,191 @@
+/*
+ * yocopp.h - C ABI of the B200 (sm_100a) YOCO / YOCO++ cross-layer KV cache
+ * hot path: the fused residual composition + cache append, and the
+ * split-K GQA decode attention that every cross-decoder layer runs over the
+ * single shared cache.
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers of the current CUDA device,
+ *    owned by the caller.  The library never allocates or frees them and
+ *    keeps no reference after the call returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL is the legacy default stream).  A YOCOPP_OK return means the work
+ *    was enqueued; it does not wait for it.
+ *  - Host-side argument checks return a negative yocopp_status and enqueue
+ *    nothing.  Nothing is thrown across the ABI.
+ *  - Values the host cannot see without synchronising (positions, lengths,
+ *    block-table entries) are checked in the kernels; a violation skips the
+ *    offending access and records a code that yocopp_get_device_status()
+ *    returns.  Kernels never trap.
+ *  - Element types: YOCOPP_BF16 (storage bf16, fp32 arithmetic) or
+ *    YOCOPP_F32.  q, K, V, the cache and the output share one type.
+ */
+#ifndef YOCOPP_H
+#define YOCOPP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum yocopp_status {
+    YOCOPP_OK = 0,
+    YOCOPP_EINVAL = -1,        /* null pointer, bad size, unsupported shape */
+    YOCOPP_EDTYPE = -2,        /* unknown or unsupported element type */
+    YOCOPP_ECAPACITY = -3,     /* a position / length beyond the cache (device check) */
+    YOCOPP_EWORKSPACE = -4,    /* workspace missing, misaligned or too small */
+    YOCOPP_ECUDA = -5,         /* a CUDA runtime/driver call failed */
+    YOCOPP_EDEVICE_CHECK = -6, /* a kernel met an invalid block-table entry */
+    YOCOPP_ETIMEOUT = -7       /* a bounded wait inside a kernel ran out */
+} yocopp_status;
+
+typedef enum yocopp_dtype {
+    YOCOPP_BF16 = 0,
+    YOCOPP_F32 = 1
+} yocopp_dtype;
+
+/*
+ * One layer's KV cache (caller-owned device memory).
+ *
+ * Contiguous (block_table == NULL):
+ *   k, v : [batch][num_kv_heads][capacity][head_dim]
+ * Paged (block_table != NULL):
+ *   k, v : [num_blocks][num_kv_heads][block_size][head_dim]
+ *   block_table : int32 [batch][max_blocks_per_seq]; position p of sequence b
+ *   lives in block block_table[b][p / block_size], slot p % block_size;
+ *   capacity must equal block_size * max_blocks_per_seq.
+ * In both layouts each (token, head) row is head_dim contiguous elements and
+ * each (sequence or block, head) plane is contiguous, which is what lets the
+ * decode kernel stage K/V tiles with TMA.
+ *
+ * Supported: head_dim in {64, 128}; block_size in {16, 32, 64, 128, 256};
+ * k and v 16-byte aligned.  In YOCO++ (section 2, "cache strategy") a
+ * self-decoder layer's cache holds the composed K'_i, V'_i; the cross-decoder
+ * layers all read layer L/2's cache, the shared cache.
+ */
+typedef struct yocopp_cache {
+    void* k;
+    void* v;
+    const int32_t* block_table;
+    int32_t dtype;               /* yocopp_dtype */
+    int32_t batch;
+    int32_t num_kv_heads;
+    int32_t head_dim;
+    int32_t capacity;            /* positions per sequence */
+    int32_t block_size;          /* paged only (ignored when contiguous) */
+    int32_t max_blocks_per_seq;  /* paged only */
+    int32_t num_blocks;          /* paged only: blocks in the pool */
+} yocopp_cache;
+
+/*
+ * yocopp_compose_append - YOCO++ residual KV composition fused with the
+ * cache write (YOCO++: Enhancing YOCO with KV Residual Connections,
+ * section 2 "method", composition equations; section 2 key innovation 1,
+ * cache strategy: the composed values are what is stored).
+ *
+ * For every new token t of sequence b, KV head h and channel c:
+ *   K'[t,h,c] = lambda * (alpha[0] * K1[t,h,c] + alpha[1] * Ki[t,h,c])
+ *   V'[t,h,c] = lambda * (alpha[2] * V1[t,h,c] + alpha[3] * Vi[t,h,c])
+ * computed in fp32 with error-free products and sums for the inner weighted
+ * sum (so near-cancelling terms keep their low bits), then multiplied by
+ * lambda, rounded once to the cache type, and written to cache positions
+ * pos[b] .. pos[b] + n_b - 1.  Stored bf16 values are within one bf16 ulp of
+ * the exact composition.
+ *
+ *   K1, V1, Ki, Vi : device, [total_new][num_kv_heads][head_dim], cache dtype,
+ *                    16-byte aligned.  Rows are token-major and packed over
+ *                    the batch: sequence b's new tokens are rows
+ *                    [cu_new[b], cu_new[b+1]) or, when cu_new == NULL,
+ *                    [b * n_uniform, (b + 1) * n_uniform).  K1/V1 are the
+ *                    current tokens' layer-1 values (they may alias Ki/Vi).
+ *   alpha          : HOST, 4 floats {aK1, aK2, aV1, aV2}.
+ *   lambda         : the scale factor (35 in the paper).
+ *   cache          : HOST descriptor of the destination cache.
+ *   pos            : device int32 [cache->batch], first position written.
+ *   cu_new         : device int32 [cache->batch + 1] prefix offsets, or NULL.
+ *   n_uniform      : tokens per sequence when cu_new == NULL (>= 0).
+ *   total_new      : number of input rows (= cu_new[batch] or batch*n_uniform).
+ *
+ * Layer 1 (raw K_1, V_1 stored) is alpha = {0, 1/lambda, 0, 1/lambda}, which
+ * reproduces the inputs bit for bit in bf16 (section 2, initialization).
+ * A row whose position is outside [0, capacity), or whose block-table entry
+ * is outside [0, num_blocks), is not written and the device status records
+ * YOCOPP_ECAPACITY / YOCOPP_EDEVICE_CHECK.  No other cache slot is touched.
+ */
+int32_t yocopp_compose_append(const void* K1, const void* V1, const void* Ki, const void* Vi,
+                              const float alpha[4], float lambda, const yocopp_cache* cache,
+                              const int32_t* pos, const int32_t* cu_new, int32_t n_uniform,
+                              int64_t total_new, void* stream);
+
+/*
+ * yocopp_decode_attn_workspace_size - bytes of device workspace that
+ * yocopp_decode_attn needs for this cache shape and query-head count on the
+ * current device (it depends on the device's SM count).  Returns a negative
+ * yocopp_status on invalid arguments.  The workspace holds the per-split
+ * partial softmax state (max, sum of exponentials, weighted value sum) and
+ * the split plan; its previous contents never matter.
+ */
+int64_t yocopp_decode_attn_workspace_size(const yocopp_cache* cache, int32_t num_q_heads);
+
+/*
+ * yocopp_decode_attn - one decode step of a cross-decoder layer over the
+ * shared cache (You Only Cache Once, abstract: the cross-decoder reuses the
+ * cached KVs through cross-attention; YOCO++ section 2: every upper-half
+ * layer reads (K'_{L/2}, V'_{L/2}); section 3: decoding reads one KV set).
+ *
+ * For sequence b and query head h with KV head g = h / (num_q_heads /
+ * num_kv_heads) (contiguous GQA grouping):
+ *   s_t = scale * <q[b,h,:], K'[b,t,g,:]>   for t in [0, seq_lens[b])
+ *   out[b,h,:] = sum_t softmax(s)_t * V'[b,t,g,:]
+ * fp32 arithmetic, online softmax over key tiles split across the GPU, then
+ * an exact log-sum-exp merge of the splits.  seq_lens[b] == 0 gives zeros.
+ *
+ *   q         : device [batch][num_q_heads][head_dim], cache dtype, 16-byte aligned.
+ *   cache     : HOST descriptor of the shared cache.
+ *   seq_lens  : device int32 [batch]; positions attended (the token being
+ *               decoded is already appended).  A length above capacity is
+ *               clamped and YOCOPP_ECAPACITY recorded on the device.
+ *   out       : device [batch][num_q_heads][head_dim], cache dtype.
+ *   num_q_heads : multiple of num_kv_heads, group size in {1, 2, 4}.
+ *   scale     : softmax scale; 0 selects 1/sqrt(head_dim).
+ *   workspace : device, >= yocopp_decode_attn_workspace_size() bytes, 256-byte
+ *               aligned, not shared with a concurrently running call.
+ */
+int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32_t* seq_lens,
+                           void* out, int32_t num_q_heads, float scale, void* workspace,
+                           int64_t workspace_bytes, void* stream);
+
+/*
+ * yocopp_get_device_status - the first error code recorded by a kernel on
+ * the current device since the last reset (YOCOPP_OK if none).  Synchronous:
+ * it waits for the device.  reset != 0 clears the record.
+ */
+int32_t yocopp_get_device_status(int32_t reset);
+
+/* Human-readable name of a yocopp_status value (static string). */
+const char* yocopp_status_string(int32_t status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int32_t yocopp_version(void);
+
+/*
+ * yocopp_testing_set_decode_fault - failure-injection hook for tests.
+ * Host-side, process-wide; affects later yocopp_decode_attn launches.
+ *   drop_tile     : index (in the split plan's flattened tile order) of one
+ *                   tile whose load is never issued, so the consumers' wait on
+ *                   it can only run out; -1 disables the injection.
+ *   wait_limit_ns : limit of every bounded wait inside the decode kernel
+ *                   (default 2 s); must be > 0.
+ * With a dropped tile the kernel records YOCOPP_ETIMEOUT, waits (bounded) for
+ * its own copies still in flight, and returns; the context stays usable.
+ * Returns YOCOPP_EINVAL for wait_limit_ns <= 0.
+ */
+int32_t yocopp_testing_set_decode_fault(int32_t drop_tile, int64_t wait_limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* YOCOPP_H */

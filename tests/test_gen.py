@@ -41,10 +41,12 @@ def test_splitmix_definition():
 def test_workloads():
     w1 = gen.config(1)
     assert (w1.batch, w1.hq, w1.hkv, w1.d, w1.dtype, w1.lens) == (1, 1, 1, 64, "f32", [256])
-    assert w1.alpha[2] == (0.1, 1 / 35 + 0.01, 0.1, 1 / 35 + 0.01) and w1.cross_layers == [3, 4]
+    f32 = lambda x: float(np.float32(x))
+    assert w1.alpha[2] == (f32(0.1), f32(1 / 35 + 0.01), f32(0.1), f32(1 / 35 + 0.01)) and w1.cross_layers == [3, 4]
     w2 = gen.config(2)
     assert w2.composed_layers == list(range(2, 13)) and w2.shared_layer == 12 and len(w2.cross_layers) == 12
     for i, a in w2.alpha.items():
+        assert all(float(np.float32(x)) == x for x in a)  # fp32-exact, as the ABI passes them
         assert abs(a[0]) <= 0.05 and abs(a[1] - 1 / 35) <= 0.05 and abs(a[2]) <= 0.05 and abs(a[3] - 1 / 35) <= 0.05
     w5 = gen.config(5)
     assert w5.batch == 64 and min(w5.lens) >= 512 and max(w5.lens) <= 32768 and w5.paged
@@ -54,7 +56,7 @@ def test_workloads():
     w4 = gen.config(4)
     pos, mode = w4.planted
     assert 0 <= pos < 131071 and mode == "aligned"
-    assert w4.alpha[12] == (0.0, 1 / 35, 0.0, 1 / 35)
+    assert w4.alpha[12] == (0.0, float(np.float32(1 / 35)), 0.0, float(np.float32(1 / 35)))
 
 
 def test_planted_row_is_aligned():
