@@ -29,7 +29,7 @@ YOCOPP_F32 = 1
 # every entry point declared in include/yocopp.h
 EXPORTS = ("yocopp_compose_append", "yocopp_decode_attn_workspace_size", "yocopp_decode_attn",
            "yocopp_get_device_status", "yocopp_status_string", "yocopp_version",
-           "yocopp_testing_set_decode_fault")
+           "yocopp_testing_set_decode_fault", "yocopp_decode_attn_static", "yocopp_decode_attn_static_capacity")
 
 
 class yocopp_cache(ctypes.Structure):
@@ -73,6 +73,10 @@ def load(path: Optional[str] = None):
     lib.yocopp_version.argtypes = []
     lib.yocopp_testing_set_decode_fault.restype = I32
     lib.yocopp_testing_set_decode_fault.argtypes = [I32, I64]
+    lib.yocopp_decode_attn_static.restype = I32
+    lib.yocopp_decode_attn_static.argtypes = [V, ctypes.POINTER(yocopp_cache), V, V, I32, ctypes.c_float, V]
+    lib.yocopp_decode_attn_static_capacity.restype = I64
+    lib.yocopp_decode_attn_static_capacity.argtypes = []
     if path is None:
         _lib = lib
     return lib
@@ -168,6 +172,20 @@ def yocopp_decode_attn(q, cache: yocopp_cache, seq_lens, out, workspace, num_q_h
                                    workspace.numel() * workspace.element_size() if workspace is not None else 0,
                                    _stream(stream))
     _check("yocopp_decode_attn", rc)
+
+
+def yocopp_decode_attn_static(q, cache: yocopp_cache, seq_lens, out, num_q_heads: Optional[int] = None,
+                              scale: float = 0.0, stream=None) -> None:
+    """yocopp_decode_attn using the library's fixed scratch array instead of a
+    caller workspace, for callers that cannot allocate device memory."""
+    hq = q.shape[1] if num_q_heads is None else num_q_heads
+    rc = load().yocopp_decode_attn_static(_ptr(q), ctypes.byref(cache), _ptr(seq_lens), _ptr(out), int(hq),
+                                          float(scale), _stream(stream))
+    _check("yocopp_decode_attn_static", rc)
+
+
+def yocopp_decode_attn_static_capacity() -> int:
+    return int(load().yocopp_decode_attn_static_capacity())
 
 
 def yocopp_get_device_status(reset: bool = False) -> int:

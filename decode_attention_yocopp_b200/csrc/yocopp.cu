@@ -183,6 +183,30 @@ int32_t check_decode_shape(const yocopp_cache* cache, int32_t num_q_heads, int* 
 }
 
 }  // namespace
+
+// ---------------------------------------------------------------- decode without allocation
+// Scratch for yocopp_decode_attn_static: a fixed device array in this library's
+// image, so callers that cannot allocate device memory still get a workspace.
+// Every device that loads the library holds it until the process exits.
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) uint8_t g_decode_scratch[kStaticScratchBytes];
+
+namespace {
+// Device address of g_decode_scratch per device, looked up once with that
+// device current (host code must not pass the symbol itself to a kernel).
+void* static_scratch_ptr(int dev) {
+    static std::mutex mu;
+    static void* ptrs[kMaxDevices] = {nullptr};
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (ptrs[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess) return nullptr;
+        ptrs[dev] = p;
+    }
+    return ptrs[dev];
+}
+}  // namespace
 }  // namespace yocopp
 
 using namespace yocopp;
@@ -345,5 +369,20 @@ int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32
     YOCOPP_DECODE_CASE(float, 64)
 #undef YOCOPP_DECODE_CASE
 }
+
+// Decode attention whose workspace is the library's own static device array
+// (no allocation anywhere).  Argument meaning as yocopp_decode_attn.
+int32_t yocopp_decode_attn_static(const void* q, const yocopp_cache* cache, const int32_t* seq_lens, void* out,
+                                  int32_t num_q_heads, float scale, void* stream) {
+    const int64_t need = yocopp_decode_attn_workspace_size(cache, num_q_heads);
+    if (need < 0) return int32_t(need);
+    if (need > int64_t(kStaticScratchBytes)) return YOCOPP_EWORKSPACE;
+    void* scratch = static_scratch_ptr(current_device());
+    if (scratch == nullptr) return YOCOPP_ECUDA;
+    return yocopp_decode_attn(q, cache, seq_lens, out, num_q_heads, scale, scratch,
+                              int64_t(kStaticScratchBytes), stream);
+}
+
+int64_t yocopp_decode_attn_static_capacity(void) { return int64_t(kStaticScratchBytes); }
 
 }  // extern "C"

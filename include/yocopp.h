@@ -158,6 +158,38 @@ int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32
                            int64_t workspace_bytes, void* stream);
 
 /*
+ * yocopp_decode_attn_static - yocopp_decode_attn without a caller workspace.
+ * The paper has no counterpart: this entry point exists for callers that
+ * cannot allocate device memory on this path, such as a host framework that
+ * owns all device memory through its own pool and gives plug-in libraries no
+ * allocator, or a serving loop in which cudaMalloc's implicit device-wide
+ * synchronisation is not acceptable.
+ *
+ * Same arguments and results as yocopp_decode_attn, minus the workspace: the
+ * split partials and the split plan live in a fixed array inside the library
+ * (4 MiB, yocopp_decode_attn_static_capacity(); every device that loads the
+ * library holds it until the process exits).  Nothing is allocated or freed
+ * by this call.
+ *   - A shape whose workspace (yocopp_decode_attn_workspace_size) exceeds
+ *     that capacity returns YOCOPP_EWORKSPACE and enqueues nothing.  At
+ *     head_dim 128 and 4 query heads per KV head that is roughly
+ *     batch * num_kv_heads <= 1800 on a 148-SM device.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents.  Nothing in it needs to start at zero (every word a call reads
+ *     is written earlier in the same call), but calls whose execution overlaps
+ *     on the GPU (different streams, or different host threads) race on it and
+ *     give wrong results: serialise them.
+ */
+int32_t yocopp_decode_attn_static(const void* q, const yocopp_cache* cache, const int32_t* seq_lens,
+                                  void* out, int32_t num_q_heads, float scale, void* stream);
+
+/* Bytes of the fixed scratch array behind yocopp_decode_attn_static. */
+int64_t yocopp_decode_attn_static_capacity(void);
+
+/*
  * yocopp_get_device_status - the first error code recorded by a kernel on
  * the current device since the last reset (YOCOPP_OK if none).  Synchronous:
  * it waits for the device.  reset != 0 clears the record.
