@@ -86,9 +86,14 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
 
-// ---- named barrier among a subset of warps ---------------------------------
-__device__ __forceinline__ void named_barrier(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+// ---- programmatic dependent launch -----------------------------------------
+// Let the dependent grid be scheduled (it still waits for this grid to finish).
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the grids this one depends on have finished and their writes are visible.
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ---- packed fp32 math (sm_100: one instruction, two lanes of fp32) --------

@@ -7,8 +7,8 @@
 // decode step is bound by HBM bandwidth on these reads.
 //
 // Work decomposition.  The (sequence, kv-head) planes are cut into TILE-token
-// tiles and flattened in (b, g, tile) order.  A persistent grid of one CTA per
-// SM takes equal contiguous ranges of that list, so any length mix is
+// tiles and flattened in (b, g, tile) order.  A persistent grid (a fixed number of CTAs
+// per SM) takes equal contiguous ranges of that list, so any length mix is
 // balanced to within one tile and each CTA streams contiguous K/V.  A CTA
 // keeps online-softmax state for the (b, g) "segment" it is in; at the end of
 // a segment it writes either the final output (segment = the whole plane) or
@@ -69,6 +69,8 @@ struct DecodeShape {
     static constexpr int TPI = 32 / CPR;                  // value phase: tokens per warp step
 };
 
+constexpr float NEG_INF_F = -INFINITY;
+
 __device__ __forceinline__ int ntiles_of(int len, int tile) { return (len + tile - 1) / tile; }
 
 __device__ __forceinline__ int clamp_len(const int32_t* lens, int b, int cap) {
@@ -124,25 +126,238 @@ struct DecodeSmem {
     static constexpr size_t kBars = kStages;                                 // full[S], empty[S], sync
     static constexpr size_t kMeta = up16(kBars + (2 * STAGES + 1) * sizeof(uint64_t));
     static constexpr size_t kP = up16(kMeta + STAGES * sizeof(TileMeta));
-    static constexpr size_t kMergeM = up16(kP + size_t(W) * TPW * G * sizeof(float));
+    static constexpr size_t kMergeM = up16(kP + size_t(W) * TPW * G * sizeof(float2));
     static constexpr size_t kMergeL = up16(kMergeM + size_t(W) * G * sizeof(float));
     static constexpr size_t kMergeO = up16(kMergeL + size_t(W) * G * sizeof(float));
     static constexpr size_t kTileStart = up16(kMergeO + size_t(W) * G * D * sizeof(float));
     static size_t bytes(int batch) { return 1024 + kTileStart + size_t(batch + 1) * sizeof(int); }
 };
 
-template <typename T, int D, int G, int W, int STAGES>
-__global__ void __launch_bounds__((W + 1) * 32, 1)
+// Per-warp state and work of a consumer warp: the group's queries in
+// registers, the online-softmax running maxima / partial sums, and the
+// running weighted value sums for this warp's share of every tile.
+template <typename T, int D, int G, int W>
+struct ConsumerWarp {
+    using S = DecodeShape<D, T>;
+    static constexpr int TILE = S::TILE, TPW = TILE / W, CPR = S::CPR, CPL = S::CPL, EPC = S::EPC, TPI = S::TPI;
+    static constexpr int QK_IT = TPW / 4;     // score steps (4 tokens per step)
+    static constexpr int PV_IT = TPW / TPI;   // value steps (TPI tokens per step)
+    static constexpr int HL = 8 / G;          // lanes holding one head's score after the reduce-scatter
+    static_assert(G == 1 || G == 2 || G == 4, "group size");
+    static_assert(TPW % 4 == 0 && TPW % TPI == 0, "tile split");
+
+    float2 q2[G][CPL * EPC / 2];  // q * scale * log2(e), this lane's channels
+    float2 acc[G][EPC / 2];       // running sum of p * v, this lane's channel chunk
+    float m_run[G];               // running maximum per head (warp-uniform)
+    float l_part;                 // running sum of p for head hr over this lane's tokens
+    float m_mine;                 // m_run[hr], kept as a scalar (an indexed read would spill the state)
+    const int warp, lane, j4, r8, hr, pc, pslot, pbx, pcc;
+
+    __device__ __forceinline__ ConsumerWarp(int warp_, int lane_)
+        : warp(warp_), lane(lane_), j4(lane_ >> 3), r8(lane_ & 7), hr((lane_ & 7) / HL), pc(lane_ % CPR),
+          pslot(lane_ / CPR), pbx((lane_ % CPR) >> 3), pcc((lane_ % CPR) & 7) {}
+
+    // New (sequence, kv-head) segment: reset the state and load the group's queries.
+    __device__ __forceinline__ void begin_segment(const DecodeParams& p, int b, int g) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            m_run[h] = NEG_INF_F;
+#pragma unroll
+            for (int e = 0; e < EPC / 2; ++e) acc[h][e] = make_float2(0.f, 0.f);
+            const uint8_t* qrow = p.q + (int64_t(b) * p.hq + g * G + h) * S::ROWB;
+#pragma unroll
+            for (int jb = 0; jb < CPL; ++jb) {
+                const uint4 v = ld_stream(qrow + (r8 + 8 * jb) * 16);
+                const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
+                if constexpr (S::EB == 2) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = bf16x2_to_float2(w[e]);
+                        q2[h][jb * 4 + e] = make_float2(f.x * p.qscale, f.y * p.qscale);
+                    }
+                } else {
+                    q2[h][jb * 2 + 0] = make_float2(__uint_as_float(w[0]) * p.qscale, __uint_as_float(w[1]) * p.qscale);
+                    q2[h][jb * 2 + 1] = make_float2(__uint_as_float(w[2]) * p.qscale, __uint_as_float(w[3]) * p.qscale);
+                }
+            }
+        }
+        l_part = 0.f;
+        m_mine = NEG_INF_F;
+    }
+
+    // Score of one token row for head hr (8 lanes per token, packed FMAs, reduce-scatter).
+    __device__ __forceinline__ float score(const uint8_t* Kt, int row) const {
+        float2 part[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) part[h] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int jb = 0; jb < CPL; ++jb) {
+            const uint4 kv = *reinterpret_cast<const uint4*>(Kt + jb * S::BOXB + row * 128 + ((r8 ^ (row & 7)) << 4));
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(&kv);
+            if constexpr (S::EB == 2) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 kf = bf16x2_to_float2(w[e]);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) part[h] = ffma2(q2[h][jb * 4 + e], kf, part[h]);
+                }
+            } else {
+                const float2 k0 = make_float2(__uint_as_float(w[0]), __uint_as_float(w[1]));
+                const float2 k1 = make_float2(__uint_as_float(w[2]), __uint_as_float(w[3]));
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    part[h] = ffma2(q2[h][jb * 2 + 0], k0, part[h]);
+                    part[h] = ffma2(q2[h][jb * 2 + 1], k1, part[h]);
+                }
+            }
+        }
+        float v[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) v[h] = part[h].x + part[h].y;
+        float sc;
+        if constexpr (G == 4) {
+            const bool up = r8 & 4;
+            float k0 = up ? v[2] : v[0], k1 = up ? v[3] : v[1];
+            const float s0 = up ? v[0] : v[2], s1 = up ? v[1] : v[3];
+            k0 += __shfl_xor_sync(0xffffffffu, s0, 4);
+            k1 += __shfl_xor_sync(0xffffffffu, s1, 4);
+            const bool up2 = r8 & 2;
+            sc = up2 ? k1 : k0;
+            sc += __shfl_xor_sync(0xffffffffu, up2 ? k0 : k1, 2);
+            sc += __shfl_xor_sync(0xffffffffu, sc, 1);
+        } else if constexpr (G == 2) {
+            const bool up = r8 & 4;
+            sc = up ? v[1] : v[0];
+            sc += __shfl_xor_sync(0xffffffffu, up ? v[0] : v[1], 4);
+            sc += __shfl_xor_sync(0xffffffffu, sc, 2);
+            sc += __shfl_xor_sync(0xffffffffu, sc, 1);
+        } else {
+            sc = v[0];
+            sc += __shfl_xor_sync(0xffffffffu, sc, 4);
+            sc += __shfl_xor_sync(0xffffffffu, sc, 2);
+            sc += __shfl_xor_sync(0xffffffffu, sc, 1);
+        }
+        return sc;
+    }
+
+    // One tile: scores, online-softmax update, values.  MASK: the slice holds
+    // tokens at or past len (the last tile of a sequence).
+    template <bool MASK>
+    __device__ __forceinline__ void tile(const uint8_t* Kt, const uint8_t* Vt, float2* p2, int tok0, int len) {
+        const int rbase = warp * TPW;
+        float s[QK_IT];
+#pragma unroll
+        for (int i = 0; i < QK_IT; ++i) {
+            s[i] = score(Kt, rbase + i * 4 + j4);
+            if (MASK && tok0 + i * 4 + j4 >= len) s[i] = NEG_INF_F;
+        }
+        // maxima of this slice per head, then the (warp-uniform) running update
+        float mloc = s[0];
+#pragma unroll
+        for (int i = 1; i < QK_IT; ++i) mloc = fmaxf(mloc, s[i]);
+        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 8));
+        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 16));
+        float mnew[G];
+        bool grow = false;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            mnew[h] = fmaxf(m_run[h], __shfl_sync(0xffffffffu, mloc, h * HL));
+            grow |= mnew[h] > m_run[h];
+        }
+        if (grow) {  // rescale only when some maximum rose
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float corr = mnew[h] == NEG_INF_F ? 1.f : exp2f(m_run[h] - mnew[h]);
+                m_run[h] = mnew[h];
+                const float2 c2 = make_float2(corr, corr);
+#pragma unroll
+                for (int e = 0; e < EPC / 2; ++e) acc[h][e] = fmul2(acc[h][e], c2);
+                if (h == hr) {
+                    l_part *= corr;
+                    m_mine = mnew[h];
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < QK_IT; ++i) {
+            const float pr = (MASK && s[i] == NEG_INF_F) ? 0.f : exp2f(s[i] - m_mine);
+            l_part += pr;
+            if (r8 % HL == 0) p2[(i * 4 + j4) * G + hr] = make_float2(pr, pr);
+        }
+        __syncwarp();
+
+        // values: acc[h] += p[h] * v over the slice (TPI tokens per step)
+#pragma unroll
+        for (int i2 = 0; i2 < PV_IT; ++i2) {
+            const int tl = i2 * TPI + pslot;  // token within the slice
+            const int tk = rbase + tl;        // row within the tile
+            uint4 vv = *reinterpret_cast<const uint4*>(Vt + pbx * S::BOXB + tk * 128 + ((pcc ^ (tk & 7)) << 4));
+            if (MASK && tok0 + tl >= len) vv = make_uint4(0u, 0u, 0u, 0u);  // never use rows past the sequence
+            float2 pp[G];
+            if constexpr (G >= 2) {
+#pragma unroll
+                for (int h = 0; h < G; h += 2) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(p2 + tl * G + h);
+                    pp[h] = make_float2(t4.x, t4.y);
+                    pp[h + 1] = make_float2(t4.z, t4.w);
+                }
+            } else {
+                pp[0] = p2[tl];
+            }
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(&vv);
+            float2 vf[EPC / 2];
+            if constexpr (S::EB == 2) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) vf[e] = bf16x2_to_float2(w[e]);
+            } else {
+                vf[0] = make_float2(__uint_as_float(w[0]), __uint_as_float(w[1]));
+                vf[1] = make_float2(__uint_as_float(w[2]), __uint_as_float(w[3]));
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+                for (int e = 0; e < EPC / 2; ++e) acc[h][e] = ffma2(pp[h], vf[e], acc[h][e]);
+        }
+        __syncwarp();  // p2 is rewritten by the next tile
+    }
+
+    // Reduce this warp's state over its lanes and store it for the CTA merge.
+    __device__ __forceinline__ void stash(float* mg_m, float* mg_l, float* mg_o) {
+        float lsum = (r8 % HL == 0) ? l_part : 0.f;
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+#pragma unroll
+        for (int o = CPR; o < 32; o <<= 1)
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+                for (int e = 0; e < EPC / 2; ++e) {
+                    acc[h][e].x += __shfl_xor_sync(0xffffffffu, acc[h][e].x, o);
+                    acc[h][e].y += __shfl_xor_sync(0xffffffffu, acc[h][e].y, o);
+                }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float lh = __shfl_sync(0xffffffffu, lsum, h * HL);
+            if (lane == 0) {
+                mg_m[warp * G + h] = m_run[h];
+                mg_l[warp * G + h] = lh;
+            }
+            if (lane < CPR) {
+#pragma unroll
+                for (int e = 0; e < EPC / 2; ++e)
+                    *reinterpret_cast<float2*>(mg_o + (warp * G + h) * D + lane * EPC + 2 * e) = acc[h][e];
+            }
+        }
+    }
+};
+
+template <typename T, int D, int G, int W, int STAGES, int CTAS_PER_SM>
+__global__ void __launch_bounds__((W + 1) * 32, CTAS_PER_SM)
 decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const DecodeParams p) {
     using S = DecodeShape<D, T>;
     using L = DecodeSmem<T, D, G, W, STAGES>;
-    constexpr int TILE = S::TILE, TPW = L::TPW, CPR = S::CPR, CPL = S::CPL, EPC = S::EPC, TPI = S::TPI;
-    constexpr int QK_IT = TPW / 4;
-    constexpr int PV_IT = TPW / TPI;
-    constexpr int HL = 8 / G;  // lanes holding one head's score after the reduce-scatter
-    static_assert(G == 1 || G == 2 || G == 4, "group size");
-    static_assert(TPW % 4 == 0 && TPW % TPI == 0, "tile split");
+    constexpr int TILE = S::TILE, TPW = L::TPW;
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_warp[32];
@@ -300,22 +515,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
 
     // ---------------------------------------------------------------------- consumers
-    const int j4 = lane >> 3;        // score phase: token slot within a step of 4
-    const int r8 = lane & 7;         // score phase: lane within the token's 8
-    const int hr = r8 / HL;          // head this lane's score belongs to
-    const int pc = lane % CPR;       // value phase: channel chunk owned
-    const int pslot = lane / CPR;    // value phase: token slot within a step
-    const int pbx = pc >> 3, pcc = pc & 7;
-
-    float2 q2[G][CPL * EPC / 2];
-    float2 acc[G][EPC / 2];
-    float m_run[G];
-    float l_part = 0.f;
-    const float NEG_INF = -INFINITY;
+    griddep_launch_dependents();  // the combine grid may be scheduled; it waits for this grid to finish
+    ConsumerWarp<T, D, G, W> cw(warp, lane);
+    float2* p2 = reinterpret_cast<float2*>(p_s) + warp * TPW * G;  // this warp's (p, p) pairs
 
     int nsync = 0;
-    // bounded rendezvous of the W consumer warps (a named barrier could not time out)
-    // (every lane waits; the warp proceeds only if all lanes saw the phase complete)
+    // bounded rendezvous of the W consumer warps (a named barrier could not time out);
+    // every lane waits and the warp proceeds only if all lanes saw the phase complete
     auto consumer_sync = [&]() -> bool {
         __syncwarp();
         if (lane == 0) mbar_arrive(sync_bar);
@@ -337,190 +543,18 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         const TileMeta mt = meta[stage];
         const uint8_t* Kt = stage_mem + size_t(stage) * S::STAGE_BYTES;
         const uint8_t* Vt = Kt + S::KV_BYTES;
-
-        if (mt.flags & kFirst) {
-            // new (sequence, kv-head) segment: reset state, load the group's queries
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                m_run[h] = NEG_INF;
-#pragma unroll
-                for (int e = 0; e < EPC / 2; ++e) acc[h][e] = make_float2(0.f, 0.f);
-                const uint8_t* qrow = p.q + (int64_t(mt.b) * p.hq + mt.g * G + h) * S::ROWB;
-#pragma unroll
-                for (int jb = 0; jb < CPL; ++jb) {
-                    const uint4 v = ld_stream(qrow + (r8 + 8 * jb) * 16);
-                    const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
-                    if constexpr (S::EB == 2) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            float2 f = bf16x2_to_float2(w[e]);
-                            q2[h][jb * 4 + e] = make_float2(f.x * p.qscale, f.y * p.qscale);
-                        }
-                    } else {
-                        q2[h][jb * 2 + 0] = make_float2(__uint_as_float(w[0]) * p.qscale, __uint_as_float(w[1]) * p.qscale);
-                        q2[h][jb * 2 + 1] = make_float2(__uint_as_float(w[2]) * p.qscale, __uint_as_float(w[3]) * p.qscale);
-                    }
-                }
-            }
-            l_part = 0.f;
-        }
-
-        // ---- scores: s = (q * scale * log2 e) . k for this warp's TPW tokens
-        float s[QK_IT];
-#pragma unroll
-        for (int i = 0; i < QK_IT; ++i) {
-            const int row = warp * TPW + i * 4 + j4;
-            float2 part[G];
-#pragma unroll
-            for (int h = 0; h < G; ++h) part[h] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int jb = 0; jb < CPL; ++jb) {
-                const uint4 kv = *reinterpret_cast<const uint4*>(Kt + jb * S::BOXB + row * 128 + ((r8 ^ (row & 7)) << 4));
-                const uint32_t* w = reinterpret_cast<const uint32_t*>(&kv);
-                if constexpr (S::EB == 2) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 kf = bf16x2_to_float2(w[e]);
-#pragma unroll
-                        for (int h = 0; h < G; ++h) part[h] = ffma2(q2[h][jb * 4 + e], kf, part[h]);
-                    }
-                } else {
-                    const float2 k0 = make_float2(__uint_as_float(w[0]), __uint_as_float(w[1]));
-                    const float2 k1 = make_float2(__uint_as_float(w[2]), __uint_as_float(w[3]));
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        part[h] = ffma2(q2[h][jb * 2 + 0], k0, part[h]);
-                        part[h] = ffma2(q2[h][jb * 2 + 1], k1, part[h]);
-                    }
-                }
-            }
-            float v[G];
-#pragma unroll
-            for (int h = 0; h < G; ++h) v[h] = part[h].x + part[h].y;
-            // reduce-scatter over the token's 8 lanes: lane r ends with head r / HL
-            float sc;
-            if constexpr (G == 4) {
-                const bool up = r8 & 4;
-                float k0 = up ? v[2] : v[0], k1 = up ? v[3] : v[1];
-                const float s0 = up ? v[0] : v[2], s1 = up ? v[1] : v[3];
-                k0 += __shfl_xor_sync(0xffffffffu, s0, 4);
-                k1 += __shfl_xor_sync(0xffffffffu, s1, 4);
-                const bool up2 = r8 & 2;
-                sc = up2 ? k1 : k0;
-                sc += __shfl_xor_sync(0xffffffffu, up2 ? k0 : k1, 2);
-                sc += __shfl_xor_sync(0xffffffffu, sc, 1);
-            } else if constexpr (G == 2) {
-                const bool up = r8 & 4;
-                sc = up ? v[1] : v[0];
-                sc += __shfl_xor_sync(0xffffffffu, up ? v[0] : v[1], 4);
-                sc += __shfl_xor_sync(0xffffffffu, sc, 2);
-                sc += __shfl_xor_sync(0xffffffffu, sc, 1);
-            } else {
-                sc = v[0];
-                sc += __shfl_xor_sync(0xffffffffu, sc, 4);
-                sc += __shfl_xor_sync(0xffffffffu, sc, 2);
-                sc += __shfl_xor_sync(0xffffffffu, sc, 1);
-            }
-            const int tok = mt.k * TILE + row;
-            s[i] = tok < mt.len ? sc : NEG_INF;
-        }
-
-        // ---- online softmax update (log2 domain)
-        float mloc = s[0];
-#pragma unroll
-        for (int i = 1; i < QK_IT; ++i) mloc = fmaxf(mloc, s[i]);
-        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 8));
-        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 16));
-        float corr[G];
-        float m_own = NEG_INF, corr_own = 1.f;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const float mt_h = __shfl_sync(0xffffffffu, mloc, h * HL);
-            const float mnew = fmaxf(m_run[h], mt_h);
-            corr[h] = mnew == NEG_INF ? 1.f : exp2f(m_run[h] - mnew);
-            m_run[h] = mnew;
-            if (h == hr) {
-                m_own = mnew;
-                corr_own = corr[h];
-            }
-        }
-        l_part *= corr_own;
-#pragma unroll
-        for (int i = 0; i < QK_IT; ++i) {
-            const float pr = s[i] == NEG_INF ? 0.f : exp2f(s[i] - m_own);
-            l_part += pr;
-            if (r8 % HL == 0) p_s[(warp * TPW + i * 4 + j4) * G + hr] = pr;
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const float2 c2 = make_float2(corr[h], corr[h]);
-#pragma unroll
-            for (int e = 0; e < EPC / 2; ++e) acc[h][e] = fmul2(acc[h][e], c2);
-        }
-        __syncwarp();
-
-        // ---- values: acc[h] += p[h] * v over this warp's tokens
-#pragma unroll
-        for (int i2 = 0; i2 < PV_IT; ++i2) {
-            const int tk = warp * TPW + i2 * TPI + pslot;
-            uint4 vv = *reinterpret_cast<const uint4*>(Vt + pbx * S::BOXB + tk * 128 + ((pcc ^ (tk & 7)) << 4));
-            if (mt.k * TILE + tk >= mt.len) vv = make_uint4(0u, 0u, 0u, 0u);  // never read past the sequence
-            float pv[G];
-            if constexpr (G == 4) {
-                const float4 t4 = *reinterpret_cast<const float4*>(p_s + tk * 4);
-                pv[0] = t4.x; pv[1] = t4.y; pv[2] = t4.z; pv[3] = t4.w;
-            } else if constexpr (G == 2) {
-                const float2 t2 = *reinterpret_cast<const float2*>(p_s + tk * 2);
-                pv[0] = t2.x; pv[1] = t2.y;
-            } else {
-                pv[0] = p_s[tk];
-            }
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(&vv);
-            float2 vf[EPC / 2];
-            if constexpr (S::EB == 2) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) vf[e] = bf16x2_to_float2(w[e]);
-            } else {
-                vf[0] = make_float2(__uint_as_float(w[0]), __uint_as_float(w[1]));
-                vf[1] = make_float2(__uint_as_float(w[2]), __uint_as_float(w[3]));
-            }
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                const float2 ph = make_float2(pv[h], pv[h]);
-#pragma unroll
-                for (int e = 0; e < EPC / 2; ++e) acc[h][e] = ffma2(ph, vf[e], acc[h][e]);
-            }
-        }
+        if (mt.flags & kFirst) cw.begin_segment(p, mt.b, mt.g);
+        const int tok0 = mt.k * TILE + warp * TPW;  // first token of this warp's slice
+        if (tok0 + TPW <= mt.len)
+            cw.template tile<false>(Kt, Vt, p2, tok0, mt.len);
+        else
+            cw.template tile<true>(Kt, Vt, p2, tok0, mt.len);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[stage]);
 
         if (mt.flags & kLast) {
             // ---- end of segment: merge the warps' states, emit output or a partial
-            float lsum = (r8 % HL == 0) ? l_part : 0.f;
-            lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
-            lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
-#pragma unroll
-            for (int o = CPR; o < 32; o <<= 1)
-#pragma unroll
-                for (int h = 0; h < G; ++h)
-#pragma unroll
-                    for (int e = 0; e < EPC / 2; ++e) {
-                        acc[h][e].x += __shfl_xor_sync(0xffffffffu, acc[h][e].x, o);
-                        acc[h][e].y += __shfl_xor_sync(0xffffffffu, acc[h][e].y, o);
-                    }
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                const float lh = __shfl_sync(0xffffffffu, lsum, h * HL);
-                if (lane == 0) {
-                    mg_m[warp * G + h] = m_run[h];
-                    mg_l[warp * G + h] = lh;
-                }
-                if (lane < CPR) {
-#pragma unroll
-                    for (int e = 0; e < EPC / 2; ++e)
-                        *reinterpret_cast<float2*>(mg_o + (warp * G + h) * D + lane * EPC + 2 * e) = acc[h][e];
-                }
-            }
+            cw.stash(mg_m, mg_l, mg_o);
             if (!consumer_sync()) {
                 record_status(YOCOPP_ETIMEOUT);
                 s_abort = 1;
@@ -529,11 +563,11 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             const int slot = mt.b * p.hkv + mt.g + int(blockIdx.x);
             for (int idx = tid; idx < G * D; idx += W * 32) {
                 const int h = idx / D, c = idx % D;
-                float M = NEG_INF;
+                float M = NEG_INF_F;
 #pragma unroll
                 for (int w2 = 0; w2 < W; ++w2) M = fmaxf(M, mg_m[w2 * G + h]);
                 float Ls = 0.f, O = 0.f;
-                if (M != NEG_INF) {
+                if (M != NEG_INF_F) {
 #pragma unroll
                     for (int w2 = 0; w2 < W; ++w2) {
                         const float f = exp2f(mg_m[w2 * G + h] - M);
@@ -567,46 +601,46 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     if (lane == 0) atomicAdd(&s_cdone, 1);
 }
 
-// Merge the partials of planes that span several CTAs; zero planes with no tokens.
+// Merge the partials of planes that span several CTAs; zero planes with no
+// tokens.  One CTA per (plane, query head of the group), one thread per
+// channel.  Launched as a programmatic dependent of the split kernel: it may
+// be resident early, and griddepcontrol.wait holds it until the split grid
+// has finished and its writes are visible.
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeParams p) {
     using S = DecodeShape<D, T>;
-    const int bg = blockIdx.x;
+    griddep_wait();
+    const int bg = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
     const int b = bg / p.hkv, g = bg % p.hkv;
     const int len = clamp_len(p.seq_lens, b, p.capacity);
     const int nt = ntiles_of(len, S::TILE);
-    const int64_t obase = (int64_t(b) * p.hq + g * G) * D;
-    if (nt == 0) {
-        for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-            if constexpr (S::EB == 2)
-                reinterpret_cast<__nv_bfloat16*>(p.out)[obase + idx] = __float2bfloat16_rn(0.f);
-            else
-                reinterpret_cast<float*>(p.out)[obase + idx] = 0.f;
-        }
-        return;
-    }
-    const int total = p.ws_tile_start[p.batch];
-    const int tpc = (total + p.num_ctas - 1) / p.num_ctas;
-    const int first = p.ws_tile_start[b] + g * nt;
-    const int c0 = first / tpc, c1 = (first + nt - 1) / tpc;
-    if (c0 == c1) return;  // the plane was finished inside one CTA
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-        const int h = idx / D, c = idx % D;
+    const int64_t oi = (int64_t(b) * p.hq + g * G + h) * D + c;
+    float y = 0.f;
+    if (nt > 0) {
+        const int total = p.ws_tile_start[p.batch];
+        const int tpc = (total + p.num_ctas - 1) / p.num_ctas;
+        const int first = p.ws_tile_start[b] + g * nt;
+        const int c0 = first / tpc, c1 = (first + nt - 1) / tpc;
+        if (c0 == c1) return;  // the plane was finished inside one CTA
+        const float* pm = p.ws_m + int64_t(bg) * G + h;
+        const float* pl = p.ws_l + int64_t(bg) * G + h;
+        const float* po = p.ws_o + (int64_t(bg) * G + h) * D + c;
         float M = -INFINITY;
-        for (int cta = c0; cta <= c1; ++cta) M = fmaxf(M, p.ws_m[int64_t(bg + cta) * G + h]);
+#pragma unroll 8
+        for (int cta = c0; cta <= c1; ++cta) M = fmaxf(M, pm[int64_t(cta) * G]);
         float Ls = 0.f, O = 0.f;
+#pragma unroll 8
         for (int cta = c0; cta <= c1; ++cta) {
-            const int64_t sl = bg + cta;
-            const float f = exp2f(p.ws_m[sl * G + h] - M);
-            Ls += f * p.ws_l[sl * G + h];
-            O += f * p.ws_o[(sl * G + h) * D + c];
+            const float f = exp2f(pm[int64_t(cta) * G] - M);
+            Ls += f * pl[int64_t(cta) * G];
+            O += f * po[int64_t(cta) * G * D];
         }
-        const float y = Ls > 0.f ? O / Ls : 0.f;
-        if constexpr (S::EB == 2)
-            reinterpret_cast<__nv_bfloat16*>(p.out)[obase + idx] = __float2bfloat16_rn(y);
-        else
-            reinterpret_cast<float*>(p.out)[obase + idx] = y;
+        y = Ls > 0.f ? O / Ls : 0.f;
     }
+    if constexpr (S::EB == 2)
+        reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(y);
+    else
+        reinterpret_cast<float*>(p.out)[oi] = y;
 }
 
 }  // namespace yocopp

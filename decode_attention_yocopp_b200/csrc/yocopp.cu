@@ -113,20 +113,33 @@ int32_t launch_compose(ComposeParams& p, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------- decode
+// Launch shape of the split kernel: consumer warps per CTA, pipeline stages,
+// CTAs per SM (compile-time; the defaults are the measured best on B200).
+#ifndef YOCOPP_DECODE_WARPS
+#define YOCOPP_DECODE_WARPS 4
+#endif
+#ifndef YOCOPP_DECODE_STAGES
+#define YOCOPP_DECODE_STAGES 3
+#endif
+#ifndef YOCOPP_DECODE_CTAS_PER_SM
+#define YOCOPP_DECODE_CTAS_PER_SM 2
+#endif
+
 struct DecodeLaunch {
-    int w, stages, tile;
+    int w, stages, tile, ctas_per_sm;
 };
 
 template <typename T, int D>
 constexpr DecodeLaunch decode_cfg() {
-    return DecodeLaunch{4, 5, DecodeShape<D, T>::TILE};
+    return DecodeLaunch{YOCOPP_DECODE_WARPS, YOCOPP_DECODE_STAGES, DecodeShape<D, T>::TILE,
+                        YOCOPP_DECODE_CTAS_PER_SM};
 }
 
 template <typename T, int D, int G>
 int32_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, cudaStream_t st) {
     constexpr DecodeLaunch cfg = decode_cfg<T, D>();
     constexpr int W = cfg.w, STAGES = cfg.stages;
-    auto kern = decode_split_kernel<T, D, G, W, STAGES>;
+    auto kern = decode_split_kernel<T, D, G, W, STAGES, cfg.ctas_per_sm>;
     const size_t smem = DecodeSmem<T, D, G, W, STAGES>::bytes(p.batch);
     static bool attr_set[kMaxDevices] = {false};
     const int dev = current_device();
@@ -147,8 +160,18 @@ int32_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const Decode
     kern<<<p.num_ctas, (W + 1) * 32, smem, st>>>(tk, tv, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return YOCOPP_ECUDA;
-    decode_combine_kernel<T, D, G><<<p.batch * p.hkv, 128, 0, st>>>(p);
-    return cuda_status(cudaGetLastError());
+    // the combine kernel is a programmatic dependent: its launch overlaps the split kernel's tail
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(unsigned(p.batch * p.hkv), unsigned(G), 1);
+    lc.blockDim = dim3(D, 1, 1);
+    lc.dynamicSmemBytes = 0;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&lc, decode_combine_kernel<T, D, G>, p));
 }
 
 struct WorkspaceLayout {
@@ -301,7 +324,8 @@ int64_t yocopp_decode_attn_workspace_size(const yocopp_cache* cache, int32_t num
     if (rc != YOCOPP_OK) return rc;
     const int sms = sm_count(current_device());
     if (sms <= 0) return YOCOPP_ECUDA;
-    return int64_t(workspace_layout(cache->batch, cache->num_kv_heads, G, cache->head_dim, sms).total);
+    return int64_t(workspace_layout(cache->batch, cache->num_kv_heads, G, cache->head_dim,
+                                    sms * YOCOPP_DECODE_CTAS_PER_SM).total);
 }
 
 int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32_t* seq_lens, void* out,
@@ -315,7 +339,8 @@ int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32
     if (!(scale >= 0.f) || !std::isfinite(scale)) return YOCOPP_EINVAL;
     const int sms = sm_count(current_device());
     if (sms <= 0) return YOCOPP_ECUDA;
-    const WorkspaceLayout wl = workspace_layout(cache->batch, cache->num_kv_heads, G, cache->head_dim, sms);
+    const int num_ctas = sms * YOCOPP_DECODE_CTAS_PER_SM;
+    const WorkspaceLayout wl = workspace_layout(cache->batch, cache->num_kv_heads, G, cache->head_dim, num_ctas);
     if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < int64_t(wl.total))
         return YOCOPP_EWORKSPACE;
 
@@ -350,7 +375,7 @@ int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32
     p.mbps = paged ? cache->max_blocks_per_seq : 0;
     p.num_blocks = paged ? cache->num_blocks : 0;
     p.boxr = boxr;
-    p.num_ctas = sms;
+    p.num_ctas = num_ctas;
     p.drop_tile = g_test_drop_tile;
     p.wait_limit_ns = g_wait_limit_ns;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
