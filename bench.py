@@ -238,7 +238,7 @@ class Step:
         self.q = {l: w.device(gen.Q, l) for l in self.cross}
         self.out = {l: torch.empty((w.batch, w.hq, w.d), dtype=self.tdt, device="cuda") for l in self.cross}
         self.prefill_ntok = w.total_prefill
-        self.launches_per_step = 2 * len(comp) + 2 * len(self.cross)
+        self.launches_per_step = 2 * len(comp) + len(self.cross)  # compose x2 per layer, one decode launch per layer
 
     def run(self, ev=None):
         """One step; ev = dict of event lists to record phase boundaries into."""
@@ -346,7 +346,7 @@ def run_ours(args, rank, world, local):
                  "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(ach_comp / peak, 4),
                  "traffic": ncu_traffic("compose_append_kernel", workload),
                  "algorithmic_bytes_per_launch": w.compose_bytes(w.total_prefill)}
-    roof_attn = {"kernel": "decode_split_kernel + decode_combine_kernel (one layer)", "bound": "hbm",
+    roof_attn = {"kernel": "decode_split_kernel (one layer, split + merge)", "bound": "hbm",
                  "achieved": round(ach_attn, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                  "frac": round(ach_attn / peak, 4), "traffic": ncu_traffic("decode_split_kernel", workload),
                  "algorithmic_bytes_per_launch": kv_bytes_layer}

@@ -29,7 +29,7 @@ YOCOPP_F32 = 1
 # every entry point declared in include/yocopp.h
 EXPORTS = ("yocopp_compose_append", "yocopp_decode_attn_workspace_size", "yocopp_decode_attn",
            "yocopp_get_device_status", "yocopp_status_string", "yocopp_version",
-           "yocopp_testing_set_decode_fault", "yocopp_decode_attn_static", "yocopp_decode_attn_static_capacity")
+           "yocopp_testing_set_decode_fault", "yocopp_decode_attn_static")
 
 
 class yocopp_cache(ctypes.Structure):
@@ -75,8 +75,6 @@ def load(path: Optional[str] = None):
     lib.yocopp_testing_set_decode_fault.argtypes = [I32, I64]
     lib.yocopp_decode_attn_static.restype = I32
     lib.yocopp_decode_attn_static.argtypes = [V, ctypes.POINTER(yocopp_cache), V, V, I32, ctypes.c_float, V]
-    lib.yocopp_decode_attn_static_capacity.restype = I64
-    lib.yocopp_decode_attn_static_capacity.argtypes = []
     if path is None:
         _lib = lib
     return lib
@@ -184,8 +182,7 @@ def yocopp_decode_attn_static(q, cache: yocopp_cache, seq_lens, out, num_q_heads
     _check("yocopp_decode_attn_static", rc)
 
 
-def yocopp_decode_attn_static_capacity() -> int:
-    return int(load().yocopp_decode_attn_static_capacity())
+STATIC_SCRATCH_BYTES = 4 << 20  # size of the library's fixed scratch array (include/yocopp.h)
 
 
 def yocopp_get_device_status(reset: bool = False) -> int:
@@ -205,7 +202,7 @@ def yocopp_testing_set_decode_fault(drop_tile: int = -1, wait_limit_ns: int = 2_
 
 
 def alloc_workspace(cache: yocopp_cache, num_q_heads: int, device=None):
-    """A torch byte tensor large enough (and 256-byte aligned) for yocopp_decode_attn."""
+    """A zero-filled torch byte tensor large enough (and 256-byte aligned) for yocopp_decode_attn."""
     import torch
     n = yocopp_decode_attn_workspace_size(cache, num_q_heads)
-    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")

@@ -13,8 +13,9 @@
 // keeps online-softmax state for the (b, g) "segment" it is in; at the end of
 // a segment it writes either the final output (segment = the whole plane) or
 // an unnormalised partial (max, sum of exponentials, weighted value sum) to a
-// workspace slot; the combine kernel merges partials of planes that span
-// several CTAs with an exact log-sum-exp.
+// workspace slot; the last CTA to finish a plane that spans several CTAs
+// (counted with an atomic arrival counter) merges its partials with an exact
+// log-sum-exp and writes the output.  One launch per layer.
 //
 // Inside a CTA.  One producer warp issues TMA tile loads (128-byte swizzled
 // boxes, so the compute warps read shared memory without bank conflicts) into
@@ -38,7 +39,7 @@ struct DecodeParams {
     uint8_t* out;
     const int32_t* seq_lens;
     const int32_t* block_table;  // nullptr: contiguous cache
-    int32_t* ws_tile_start;      // [batch + 1]
+    unsigned long long* ws_cnt;  // [batch * hkv] arrival counters: (call epoch << 20) | CTAs arrived
     float* ws_m;                 // [slots][G]
     float* ws_l;                 // [slots][G]
     float* ws_o;                 // [slots][G][D]
@@ -47,6 +48,7 @@ struct DecodeParams {
     int32_t num_ctas;
     int32_t drop_tile;           // testing: a tile whose load is never issued (-1: none)
     uint64_t wait_limit_ns;
+    unsigned long long epoch;    // grows with every call (44 bits, never 0): tags this call's arrivals
 };
 
 struct TileMeta {
@@ -70,6 +72,14 @@ struct DecodeShape {
 };
 
 constexpr float NEG_INF_F = -INFINITY;
+
+template <typename T>
+__device__ __forceinline__ void write_out(uint8_t* out, int64_t i, float y) {
+    if constexpr (sizeof(T) == 2)
+        reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(y);
+    else
+        reinterpret_cast<float*>(out)[i] = y;
+}
 
 __device__ __forceinline__ int ntiles_of(int len, int tile) { return (len + tile - 1) / tile; }
 
@@ -132,6 +142,19 @@ struct DecodeSmem {
     static constexpr size_t kTileStart = up16(kMergeO + size_t(W) * G * D * sizeof(float));
     static size_t bytes(int batch) { return 1024 + kTileStart + size_t(batch + 1) * sizeof(int); }
 };
+
+// Arrive on a plane's counter for this call; returns how many CTAs have arrived
+// (this one included), or 0 if the counter holds a later call's tag (a
+// workspace that was not zero-filled before its first use).  The word is
+// (epoch << 20) | count.  Epochs only grow within a process, so atomicMax
+// replaces a tag left by any earlier call (finished or aborted) with this
+// call's tag and a zero count; two single atomics, no retry loop.
+__device__ __forceinline__ unsigned arrive_plane(unsigned long long* cnt, unsigned long long epoch) {
+    atomicMax(cnt, epoch << 20);
+    const unsigned long long old = atomicAdd(cnt, 1ull);
+    if ((old >> 20) != epoch) return 0;
+    return unsigned(old & 0xFFFFFull) + 1u;
+}
 
 // Per-warp state and work of a consumer warp: the group's queries in
 // registers, the online-softmax running maxima / partial sums, and the
@@ -351,6 +374,80 @@ struct ConsumerWarp {
     }
 };
 
+// Merge the partials of one (sequence, kv-head) plane written by CTAs c0..c1
+// (slots plane + cta) and write the group's outputs.  Run by the W consumer
+// warps of the last CTA to arrive.  One parallel pass stages every part's
+// maximum and sum in shared memory (the probability and warp-merge areas,
+// free at this point); weights e^{m_s - M} are formed once per (part, head);
+// then each thread accumulates 4 channels with 16-byte loads.
+template <typename T, int D, int G, int W, typename Sync>
+__device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c0, int c1, int64_t out_row0,
+                                            float* scratch, int scratch_floats, Sync& sync) {
+    constexpr int NT = W * 32;
+    const int tid = threadIdx.x;
+    const int nparts = c1 - c0 + 1;
+    const int cap = (scratch_floats - 2 * G) / (2 * G);  // parts that fit the staging area
+    const float* pm = p.ws_m + int64_t(bg + c0) * G;
+    const float* pl = p.ws_l + int64_t(bg + c0) * G;
+    const float4* po = reinterpret_cast<const float4*>(p.ws_o + int64_t(bg + c0) * G * D);
+    if (nparts > cap) {
+        // very many splits of one plane: per-element loop without staging
+        for (int idx = tid; idx < G * D; idx += NT) {
+            const int h = idx / D, c = idx % D;
+            float M = NEG_INF_F;
+            for (int s2 = 0; s2 < nparts; ++s2) M = fmaxf(M, __ldcg(pm + s2 * G + h));
+            float Ls = 0.f, O = 0.f;
+            for (int s2 = 0; s2 < nparts; ++s2) {
+                const float f = exp2f(__ldcg(pm + s2 * G + h) - M);
+                Ls += f * __ldcg(pl + s2 * G + h);
+                O += f * __ldcg(p.ws_o + (int64_t(bg + c0 + s2) * G + h) * D + c);
+            }
+            write_out<T>(p.out, out_row0 * D + idx, Ls > 0.f ? O / Ls : 0.f);
+        }
+        return true;
+    }
+    float* wts = scratch;                   // [part][G]: maxima, then weights
+    float* lss = scratch + cap * G;         // [part][G]: sums of exponentials
+    float* Mh = scratch + 2 * cap * G;      // [G] maxima, [G] normalisers
+    for (int i = tid; i < nparts * G; i += NT) {
+        wts[i] = __ldcg(pm + i);
+        lss[i] = __ldcg(pl + i);
+    }
+    bool ok = sync();
+    if (tid < G) {
+        float M = NEG_INF_F;
+        for (int s2 = 0; s2 < nparts; ++s2) M = fmaxf(M, wts[s2 * G + tid]);
+        Mh[tid] = M;
+    }
+    ok = sync() && ok;
+    for (int i = tid; i < nparts * G; i += NT) wts[i] = exp2f(wts[i] - Mh[i % G]);
+    ok = sync() && ok;
+    if (tid < G) {
+        float Ls = 0.f;
+        for (int s2 = 0; s2 < nparts; ++s2) Ls += wts[s2 * G + tid] * lss[s2 * G + tid];
+        Mh[G + tid] = Ls;
+    }
+    ok = sync() && ok;
+    for (int q4 = tid; q4 < G * D / 4; q4 += NT) {
+        const int h = (q4 * 4) / D;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int s2 = 0; s2 < nparts; ++s2) {
+            const float4 o = __ldcg(po + int64_t(s2) * (G * D / 4) + q4);
+            const float f = wts[s2 * G + h];
+            O.x += f * o.x; O.y += f * o.y; O.z += f * o.z; O.w += f * o.w;
+        }
+        const float Ls = Mh[G + h];
+        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+        const int64_t o0 = out_row0 * D + int64_t(q4) * 4;
+        write_out<T>(p.out, o0 + 0, O.x * inv);
+        write_out<T>(p.out, o0 + 1, O.y * inv);
+        write_out<T>(p.out, o0 + 2, O.z * inv);
+        write_out<T>(p.out, o0 + 3, O.w * inv);
+    }
+    return ok;
+}
+
 template <typename T, int D, int G, int W, int STAGES, int CTAS_PER_SM>
 __global__ void __launch_bounds__((W + 1) * 32, CTAS_PER_SM)
 decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -387,9 +484,18 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         s_abort = 0;
         s_cdone = 0;
     }
+    // launched as a programmatic dependent: inputs may still be in flight
+    // from the previous kernel until this wait returns
+    griddep_wait();
+    griddep_launch_dependents();
     tile_prefix<TILE>(p, s_ts, s_warp);  // ends with __syncthreads()
-    if (blockIdx.x == 0)
-        for (int b = tid; b <= p.batch; b += blockDim.x) p.ws_tile_start[b] = s_ts[b];
+    // sequences with no cached positions: zero output (CTA b mod grid writes it)
+    for (int b = blockIdx.x; b < p.batch; b += p.num_ctas) {
+        if (s_ts[b + 1] != s_ts[b]) continue;
+        for (int idx = tid; idx < p.hq * D; idx += blockDim.x) {
+            write_out<T>(p.out, int64_t(b) * p.hq * D + idx, 0.f);
+        }
+    }
 
     const int total = s_ts[p.batch];
     const int tpc = (total + p.num_ctas - 1) / p.num_ctas;
@@ -515,8 +621,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
 
     // ---------------------------------------------------------------------- consumers
-    griddep_launch_dependents();  // the combine grid may be scheduled; it waits for this grid to finish
     ConsumerWarp<T, D, G, W> cw(warp, lane);
+    __shared__ int s_last;
     float2* p2 = reinterpret_cast<float2*>(p_s) + warp * TPW * G;  // this warp's (p, p) pairs
 
     int nsync = 0;
@@ -560,7 +666,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                 s_abort = 1;
                 break;
             }
-            const int slot = mt.b * p.hkv + mt.g + int(blockIdx.x);
+            const int bg = mt.b * p.hkv + mt.g;
+            const int slot = bg + int(blockIdx.x);
+            const bool whole = mt.flags & kWhole;
             for (int idx = tid; idx < G * D; idx += W * 32) {
                 const int h = idx / D, c = idx % D;
                 float M = NEG_INF_F;
@@ -575,18 +683,44 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                         O += f * mg_o[(w2 * G + h) * D + c];
                     }
                 }
-                if (mt.flags & kWhole) {
-                    const float y = Ls > 0.f ? O / Ls : 0.f;
-                    const int64_t oi = (int64_t(mt.b) * p.hq + mt.g * G + h) * D + c;
-                    if constexpr (S::EB == 2)
-                        reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(y);
-                    else
-                        reinterpret_cast<float*>(p.out)[oi] = y;
+                if (whole) {
+                    write_out<T>(p.out, (int64_t(mt.b) * p.hq + mt.g * G + h) * D + c, Ls > 0.f ? O / Ls : 0.f);
                 } else {
                     p.ws_o[(int64_t(slot) * G + h) * D + c] = O;
                     if (c == 0) {
                         p.ws_m[int64_t(slot) * G + h] = M;
                         p.ws_l[int64_t(slot) * G + h] = Ls;
+                    }
+                }
+            }
+            if (!whole) {
+                // publish this CTA's partial, count arrivals; the last CTA merges the plane
+                __threadfence();
+                if (!consumer_sync()) {
+                    record_status(YOCOPP_ETIMEOUT);
+                    s_abort = 1;
+                    break;
+                }
+                const int nt = ntiles_of(mt.len, TILE);
+                const int first = s_ts[mt.b] + mt.g * nt;
+                const int c0 = first / tpc, c1 = (first + nt - 1) / tpc;
+                if (tid == 0) {
+                    const unsigned arrived = arrive_plane(p.ws_cnt + bg, p.epoch);
+                    if (arrived == 0) record_status(YOCOPP_EWORKSPACE);
+                    s_last = arrived == unsigned(c1 - c0 + 1);
+                    __threadfence();
+                }
+                if (!consumer_sync()) {
+                    record_status(YOCOPP_ETIMEOUT);
+                    s_abort = 1;
+                    break;
+                }
+                if (s_last) {
+                    if (!merge_plane<T, D, G, W>(p, bg, c0, c1, int64_t(mt.b) * p.hq + mt.g * G, p_s,
+                                                 int((L::kTileStart - L::kP) / sizeof(float)), consumer_sync)) {
+                        record_status(YOCOPP_ETIMEOUT);
+                        s_abort = 1;
+                        break;
                     }
                 }
             }
@@ -599,48 +733,6 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
     __syncwarp();
     if (lane == 0) atomicAdd(&s_cdone, 1);
-}
-
-// Merge the partials of planes that span several CTAs; zero planes with no
-// tokens.  One CTA per (plane, query head of the group), one thread per
-// channel.  Launched as a programmatic dependent of the split kernel: it may
-// be resident early, and griddepcontrol.wait holds it until the split grid
-// has finished and its writes are visible.
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeParams p) {
-    using S = DecodeShape<D, T>;
-    griddep_wait();
-    const int bg = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
-    const int b = bg / p.hkv, g = bg % p.hkv;
-    const int len = clamp_len(p.seq_lens, b, p.capacity);
-    const int nt = ntiles_of(len, S::TILE);
-    const int64_t oi = (int64_t(b) * p.hq + g * G + h) * D + c;
-    float y = 0.f;
-    if (nt > 0) {
-        const int total = p.ws_tile_start[p.batch];
-        const int tpc = (total + p.num_ctas - 1) / p.num_ctas;
-        const int first = p.ws_tile_start[b] + g * nt;
-        const int c0 = first / tpc, c1 = (first + nt - 1) / tpc;
-        if (c0 == c1) return;  // the plane was finished inside one CTA
-        const float* pm = p.ws_m + int64_t(bg) * G + h;
-        const float* pl = p.ws_l + int64_t(bg) * G + h;
-        const float* po = p.ws_o + (int64_t(bg) * G + h) * D + c;
-        float M = -INFINITY;
-#pragma unroll 8
-        for (int cta = c0; cta <= c1; ++cta) M = fmaxf(M, pm[int64_t(cta) * G]);
-        float Ls = 0.f, O = 0.f;
-#pragma unroll 8
-        for (int cta = c0; cta <= c1; ++cta) {
-            const float f = exp2f(pm[int64_t(cta) * G] - M);
-            Ls += f * pl[int64_t(cta) * G];
-            O += f * po[int64_t(cta) * G * D];
-        }
-        y = Ls > 0.f ? O / Ls : 0.f;
-    }
-    if constexpr (S::EB == 2)
-        reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(y);
-    else
-        reinterpret_cast<float*>(p.out)[oi] = y;
 }
 
 }  // namespace yocopp

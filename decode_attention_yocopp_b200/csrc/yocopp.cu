@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -19,6 +20,14 @@ constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
 
 int g_test_drop_tile = -1;
+
+// Per-call tag for the decode kernel's arrival counters: strictly increasing
+// within the process, 44 bits, never 0 (a zero-filled counter is older than
+// every call).
+unsigned long long next_epoch() {
+    static std::atomic<unsigned long long> counter{0};
+    return (counter.fetch_add(1) + 1) & 0xFFFFFFFFFFFull;
+}
 uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -157,25 +166,23 @@ int32_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const Decode
         attr_set[dev] = true;
     }
     if (smem > max_dyn[dev]) return YOCOPP_EINVAL;  // batch too large for the shared-memory plan
-    kern<<<p.num_ctas, (W + 1) * 32, smem, st>>>(tk, tv, p);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return YOCOPP_ECUDA;
-    // the combine kernel is a programmatic dependent: its launch overlaps the split kernel's tail
+    // launched as a programmatic dependent of the previous kernel in the stream:
+    // its launch and prologue overlap that kernel's tail (it waits before reading inputs)
     cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3(unsigned(p.batch * p.hkv), unsigned(G), 1);
-    lc.blockDim = dim3(D, 1, 1);
-    lc.dynamicSmemBytes = 0;
+    lc.gridDim = dim3(unsigned(p.num_ctas), 1, 1);
+    lc.blockDim = dim3((W + 1) * 32, 1, 1);
+    lc.dynamicSmemBytes = smem;
     lc.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
     lc.numAttrs = 1;
-    return cuda_status(cudaLaunchKernelEx(&lc, decode_combine_kernel<T, D, G>, p));
+    return cuda_status(cudaLaunchKernelEx(&lc, kern, tk, tv, p));
 }
 
 struct WorkspaceLayout {
-    size_t tile_start, m, l, o, total;
+    size_t cnt, m, l, o, total;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -183,8 +190,8 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 WorkspaceLayout workspace_layout(int batch, int hkv, int G, int D, int num_ctas) {
     const size_t slots = size_t(num_ctas) + size_t(batch) * hkv;
     WorkspaceLayout w;
-    w.tile_start = 0;
-    w.m = up256(size_t(batch + 1) * sizeof(int));
+    w.cnt = 0;
+    w.m = up256(size_t(batch) * hkv * sizeof(unsigned long long));
     w.l = w.m + up256(slots * G * sizeof(float));
     w.o = w.l + up256(slots * G * sizeof(float));
     w.total = w.o + up256(slots * G * D * sizeof(float));
@@ -361,7 +368,7 @@ int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32
     p.out = static_cast<uint8_t*>(out);
     p.seq_lens = seq_lens;
     p.block_table = cache->block_table;
-    p.ws_tile_start = reinterpret_cast<int32_t*>(ws + wl.tile_start);
+    p.ws_cnt = reinterpret_cast<unsigned long long*>(ws + wl.cnt);
     p.ws_m = reinterpret_cast<float*>(ws + wl.m);
     p.ws_l = reinterpret_cast<float*>(ws + wl.l);
     p.ws_o = reinterpret_cast<float*>(ws + wl.o);
@@ -378,6 +385,7 @@ int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32
     p.num_ctas = num_ctas;
     p.drop_tile = g_test_drop_tile;
     p.wait_limit_ns = g_wait_limit_ns;
+    p.epoch = next_epoch();
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
 #define YOCOPP_DECODE_CASE(TT, DD)                                             \
@@ -408,6 +416,5 @@ int32_t yocopp_decode_attn_static(const void* q, const yocopp_cache* cache, cons
                               int64_t(kStaticScratchBytes), stream);
 }
 
-int64_t yocopp_decode_attn_static_capacity(void) { return int64_t(kStaticScratchBytes); }
 
 }  // extern "C"

@@ -124,8 +124,12 @@ int32_t yocopp_compose_append(const void* K1, const void* V1, const void* Ki, co
  * yocopp_decode_attn needs for this cache shape and query-head count on the
  * current device (it depends on the device's SM count).  Returns a negative
  * yocopp_status on invalid arguments.  The workspace holds the per-split
- * partial softmax state (max, sum of exponentials, weighted value sum) and
- * the split plan; its previous contents never matter.
+ * partial softmax state (max, sum of exponentials, weighted value sum) and a
+ * per-(sequence, kv-head) arrival counter tagged with a per-call value that
+ * grows with every call.  Zero-fill the workspace once before its first use;
+ * after that it never needs clearing, also not after a failed call.  (A
+ * workspace that was never zero-filled can make a call report
+ * YOCOPP_EWORKSPACE through yocopp_get_device_status.)
  */
 int64_t yocopp_decode_attn_workspace_size(const yocopp_cache* cache, int32_t num_q_heads);
 
@@ -140,7 +144,10 @@ int64_t yocopp_decode_attn_workspace_size(const yocopp_cache* cache, int32_t num
  *   s_t = scale * <q[b,h,:], K'[b,t,g,:]>   for t in [0, seq_lens[b])
  *   out[b,h,:] = sum_t softmax(s)_t * V'[b,t,g,:]
  * fp32 arithmetic, online softmax over key tiles split across the GPU, then
- * an exact log-sum-exp merge of the splits.  seq_lens[b] == 0 gives zeros.
+ * an exact log-sum-exp merge of the splits by the last CTA to finish each
+ * (sequence, kv-head) plane: one kernel launch.  seq_lens[b] == 0 gives zeros.
+ * The kernel is launched as a programmatic dependent of the previous work in
+ * the stream (it waits for that work before reading any input).
  *
  *   q         : device [batch][num_q_heads][head_dim], cache dtype, 16-byte aligned.
  *   cache     : HOST descriptor of the shared cache.
@@ -166,10 +173,9 @@ int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32
  * synchronisation is not acceptable.
  *
  * Same arguments and results as yocopp_decode_attn, minus the workspace: the
- * split partials and the split plan live in a fixed array inside the library
- * (4 MiB, yocopp_decode_attn_static_capacity(); every device that loads the
- * library holds it until the process exits).  Nothing is allocated or freed
- * by this call.
+ * split partials and arrival counters live in a fixed 4 MiB array inside the
+ * library (every device that loads the library holds it until the process
+ * exits).  Nothing is allocated or freed by this call.
  *   - A shape whose workspace (yocopp_decode_attn_workspace_size) exceeds
  *     that capacity returns YOCOPP_EWORKSPACE and enqueues nothing.  At
  *     head_dim 128 and 4 query heads per KV head that is roughly
@@ -178,16 +184,14 @@ int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32
  *     (cudaGetSymbolAddress with that device current); make that first call
  *     before any stream capture.
  *   - All calls on a device share the one array and it keeps the last call's
- *     contents.  Nothing in it needs to start at zero (every word a call reads
- *     is written earlier in the same call), but calls whose execution overlaps
- *     on the GPU (different streams, or different host threads) race on it and
- *     give wrong results: serialise them.
+ *     contents.  It starts zero-filled when the library is loaded, and every
+ *     call (also a failed one) leaves it usable by the next, so nothing ever
+ *     needs clearing.  Calls whose execution overlaps on the GPU (different
+ *     streams, or different host threads) race on it and give wrong results:
+ *     serialise them.
  */
 int32_t yocopp_decode_attn_static(const void* q, const yocopp_cache* cache, const int32_t* seq_lens,
                                   void* out, int32_t num_q_heads, float scale, void* stream);
-
-/* Bytes of the fixed scratch array behind yocopp_decode_attn_static. */
-int64_t yocopp_decode_attn_static_capacity(void);
 
 /*
  * yocopp_get_device_status - the first error code recorded by a kernel on

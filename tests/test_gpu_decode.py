@@ -189,3 +189,30 @@ def test_host_errors(y):
     with pytest.raises(y.YocoppError) as e:
         y.yocopp_decode_attn(q, cache, lens, q.clone(), y.alloc_workspace(cache, 4), num_q_heads=3)
     assert e.value.status == y.YOCOPP_EINVAL
+
+
+def test_unzeroed_workspace_is_reported(y):
+    """A workspace that was never zero-filled (all bytes 0xFF: a counter tag from
+    the future) is reported as YOCOPP_EWORKSPACE; zero-filling it restores
+    correct results, and later calls never need clearing again."""
+    d, hkv, G, T = 128, 2, 4, 20000  # long enough that every plane spans several CTAs
+    k = torch.empty((1, hkv, T, d), dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    k.normal_()
+    v.normal_()
+    q = torch.randn((1, hkv * G, d), device="cuda").to(torch.bfloat16)
+    cache = y.make_cache(k, v)
+    ws = y.alloc_workspace(cache, hkv * G)
+    lens = torch.full((1,), T, dtype=torch.int32, device="cuda")
+    ref = torch.empty_like(q)
+    y.yocopp_decode_attn(q, cache, lens, ref, ws)
+    assert y.yocopp_get_device_status(reset=True) == 0
+    ws.fill_(0xFF)
+    out = torch.empty_like(q)
+    y.yocopp_decode_attn(q, cache, lens, out, ws)
+    assert y.yocopp_get_device_status(reset=True) == y.YOCOPP_EWORKSPACE
+    ws.zero_()
+    for _ in range(3):
+        y.yocopp_decode_attn(q, cache, lens, out, ws)
+        assert y.yocopp_get_device_status(reset=True) == 0
+        assert torch.equal(out, ref)

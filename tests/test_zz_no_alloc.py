@@ -75,7 +75,7 @@ def test_static_matches_workspace_twice():
 
 def test_static_rejects_oversized_shape():
     import decode_attention_yocopp_b200 as y
-    cap = y.yocopp_decode_attn_static_capacity()
+    cap = y.STATIC_SCRATCH_BYTES
     assert cap == 4 << 20
     k = torch.zeros((1, 8, 64, 128), dtype=torch.bfloat16, device="cuda")
     cache = y.make_cache(k, k, batch=4096, capacity=64)  # descriptor only: rejected before any launch
