@@ -219,14 +219,15 @@ class Step:
         comp = comp if comp is not None else w.composed_layers
         self.comp = comp
         self.cross = cross if cross is not None else w.cross_layers
+        self.selfl = [1] + comp  # self-decoder layers whose own caches the full decode step reads
         if w.paged:
             self.bt = torch.from_numpy(w.block_table()).cuda()
             self.stack = SharedKVStack(w.layers, w.batch, w.hq, w.hkv, w.d, self.tdt, w.alpha, w.lam,
                                        block_table=self.bt, block_size=w.block_size, num_blocks=w.num_blocks,
-                                       cache_layers=comp)
+                                       cache_layers=[1] + comp)
         else:
             self.stack = SharedKVStack(w.layers, w.batch, w.hq, w.hkv, w.d, self.tdt, w.alpha, w.lam,
-                                       capacity=w.max_len, cache_layers=comp)
+                                       capacity=w.max_len, cache_layers=[1] + comp)
         self.lens = torch.tensor(w.lens, dtype=torch.int32, device="cuda")
         self.pos0 = torch.zeros(w.batch, dtype=torch.int32, device="cuda")
         self.posn = torch.clamp(self.lens - 1, min=0)
@@ -235,10 +236,36 @@ class Step:
         self.vp = {i: w.device(gen.V_PREFILL, i) for i in [1] + comp}
         self.kn = {i: w.device(gen.K_NEW, i) for i in [1] + comp}
         self.vn = {i: w.device(gen.V_NEW, i) for i in [1] + comp}
-        self.q = {l: w.device(gen.Q, l) for l in self.cross}
+        self.q = {l: w.device(gen.Q, l) for l in self.cross + self.selfl}
+        self.out_self = {i: torch.empty((w.batch, w.hq, w.d), dtype=self.tdt, device="cuda") for i in self.selfl}
         self.out = {l: torch.empty((w.batch, w.hq, w.d), dtype=self.tdt, device="cuda") for l in self.cross}
         self.prefill_ntok = w.total_prefill
         self.launches_per_step = 2 * len(comp) + len(self.cross)  # compose x2 per layer, one decode launch per layer
+
+    def write_layer1_prefill(self):
+        """Layer 1 stores its raw K_1, V_1 (set up once; the composed layers are written every step)."""
+        w, s = self.w, self.stack
+        if self.cu is None:
+            s.write(1, self.kp[1], self.vp[1], self.kp[1], self.vp[1], self.pos0, n_uniform=w.lens[0] - 1)
+        else:
+            s.write(1, self.kp[1], self.vp[1], self.kp[1], self.vp[1], self.pos0, cu_new=self.cu)
+
+    def run_decode_full(self, ev=None):
+        """The attention side of one whole decode step: the decoded token appended to every
+        self-decoder layer (layer 1 raw, layers 2..L/2 composed), every self-decoder layer
+        attending over its own cache, every cross-decoder layer over the shared cache."""
+        w, s = self.w, self.stack
+        rec = (lambda k: ev[k].append(_event())) if ev is not None else (lambda k: None)
+        rec("a")
+        for i in self.selfl:
+            s.write(i, self.kn[1], self.vn[1], self.kn[i], self.vn[i], self.posn, n_uniform=1)
+        rec("b")
+        for i in self.selfl:
+            s.self_attend(i, self.q[i], self.lens, self.out_self[i])
+        rec("c")
+        for l in self.cross:
+            s.cross_attend(self.q[l], self.lens, self.out[l])
+        rec("d")
 
     def run(self, ev=None):
         """One step; ev = dict of event lists to record phase boundaries into."""
@@ -321,6 +348,22 @@ def run_ours(args, rank, world, local):
     comp_all = sum_over_ranks(comp_bytes, world)
     tok_all = sum_over_ranks(w.batch * K, world)
 
+    # the full attention-side decode step (self-decoder layers included), after the main timing
+    step.write_layer1_prefill()
+    for _ in range(2):
+        step.run_decode_full()
+    torch.cuda.synchronize()
+    evf = {k: [] for k in "abcd"}
+    barrier(world)
+    for _ in range(args.steps):
+        step.run_decode_full(evf)
+    torch.cuda.synchronize()
+    t_full = sum(a.elapsed_time(b) for a, b in zip(evf["a"], evf["d"]))
+    t_self = sum(a.elapsed_time(b) for a, b in zip(evf["b"], evf["c"]))
+    t_full_max = max_over_ranks(t_full, world)
+    t_self_max = max_over_ranks(t_self, world)
+    self_bytes = sum_over_ranks(w.kv_bytes() * len(step.selfl) * K, world)
+
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, step, world)
@@ -364,6 +407,11 @@ def run_ours(args, rank, world, local):
         "compose_frac_of_peak": round(compose_gbs / world / peak, 4),
         "decode_tok_s": round(tok_all / (t_decode_max * 1e-3), 1),
         "decode_compose_us_per_layer": round(1e3 * t_dcomp / (K * len(comp_layers)), 2),
+        "decode_full_step": {"tok_s": round(tok_all / (t_full_max * 1e-3), 1),
+                             "ms_per_step": round(t_full_max / K, 4),
+                             "self_attn_kv_gbs": round(self_bytes / (t_self_max * 1e-3) / 1e9, 1),
+                             "what": "decoded token appended to layers 1..L/2, L/2 self-decoder attentions over "
+                                     "their own caches, L/2 cross-decoder attentions over the shared cache"},
         "roofline": dominant,
         "profiling_trim": bool(args.compose_layers or args.cross_layers),
         "roofline_attention": roof_attn,

@@ -29,7 +29,8 @@ YOCOPP_F32 = 1
 # every entry point declared in include/yocopp.h
 EXPORTS = ("yocopp_compose_append", "yocopp_decode_attn_workspace_size", "yocopp_decode_attn",
            "yocopp_get_device_status", "yocopp_status_string", "yocopp_version",
-           "yocopp_testing_set_decode_fault", "yocopp_decode_attn_static")
+           "yocopp_testing_set_decode_fault", "yocopp_decode_attn_static", "yocopp_decode_attn_partial",
+           "yocopp_decode_combine")
 
 
 class yocopp_cache(ctypes.Structure):
@@ -73,6 +74,10 @@ def load(path: Optional[str] = None):
     lib.yocopp_version.argtypes = []
     lib.yocopp_testing_set_decode_fault.restype = I32
     lib.yocopp_testing_set_decode_fault.argtypes = [I32, I64]
+    lib.yocopp_decode_attn_partial.restype = I32
+    lib.yocopp_decode_attn_partial.argtypes = [V, ctypes.POINTER(yocopp_cache), V, V, I32, ctypes.c_float, V, I64, V]
+    lib.yocopp_decode_combine.restype = I32
+    lib.yocopp_decode_combine.argtypes = [V, I32, I64, I32, I32, V, V]
     lib.yocopp_decode_attn_static.restype = I32
     lib.yocopp_decode_attn_static.argtypes = [V, ctypes.POINTER(yocopp_cache), V, V, I32, ctypes.c_float, V]
     if path is None:
@@ -170,6 +175,28 @@ def yocopp_decode_attn(q, cache: yocopp_cache, seq_lens, out, workspace, num_q_h
                                    workspace.numel() * workspace.element_size() if workspace is not None else 0,
                                    _stream(stream))
     _check("yocopp_decode_attn", rc)
+
+
+def yocopp_decode_attn_partial(q, cache: yocopp_cache, seq_lens, partial, workspace, num_q_heads: Optional[int] = None,
+                               scale: float = 0.0, stream=None) -> None:
+    """Unnormalised decode attention over this cache's positions: partial is fp32
+    [batch][hq][d + 2] holding (o, m, l) per row (base-2 logits)."""
+    hq = q.shape[1] if num_q_heads is None else num_q_heads
+    rc = load().yocopp_decode_attn_partial(_ptr(q), ctypes.byref(cache), _ptr(seq_lens), _ptr(partial), int(hq),
+                                           float(scale), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size() if workspace is not None else 0,
+                                           _stream(stream))
+    _check("yocopp_decode_attn_partial", rc)
+
+
+def yocopp_decode_combine(partials, out, stream=None) -> None:
+    """Merge partials [R][..., d + 2] (fp32) into out [..., d] (bf16 or fp32)."""
+    R = partials.shape[0]
+    d = out.shape[-1]
+    rows = out.numel() // d
+    rc = load().yocopp_decode_combine(_ptr(partials), int(R), int(rows), int(d), _dtype_code(out), _ptr(out),
+                                      _stream(stream))
+    _check("yocopp_decode_combine", rc)
 
 
 def yocopp_decode_attn_static(q, cache: yocopp_cache, seq_lens, out, num_q_heads: Optional[int] = None,

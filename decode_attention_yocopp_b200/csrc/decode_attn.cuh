@@ -49,6 +49,7 @@ struct DecodeParams {
     int32_t drop_tile;           // testing: a tile whose load is never issued (-1: none)
     uint64_t wait_limit_ns;
     unsigned long long epoch;    // grows with every call (44 bits, never 0): tags this call's arrivals
+    float* part_out;             // non-null: write unnormalised [batch][hq][D + 2] (o, m, l) instead of out
 };
 
 struct TileMeta {
@@ -72,6 +73,27 @@ struct DecodeShape {
 };
 
 constexpr float NEG_INF_F = -INFINITY;
+
+// Final result of one (sequence, query head, channel): the normalised output,
+// or (partial mode) the unnormalised weighted sum plus, at channel 0, the
+// head's maximum (log2 units) and sum of exponentials.
+template <typename T, int D>
+__device__ __forceinline__ void emit(const DecodeParams& p, int64_t row, int c, float M, float Ls, float O) {
+    if (p.part_out != nullptr) {
+        float* r = p.part_out + row * (D + 2);
+        r[c] = O;
+        if (c == 0) {
+            r[D] = M;
+            r[D + 1] = Ls;
+        }
+        return;
+    }
+    const float y = Ls > 0.f ? O / Ls : 0.f;
+    if constexpr (sizeof(T) == 2)
+        reinterpret_cast<__nv_bfloat16*>(p.out)[row * D + c] = __float2bfloat16_rn(y);
+    else
+        reinterpret_cast<float*>(p.out)[row * D + c] = y;
+}
 
 template <typename T>
 __device__ __forceinline__ void write_out(uint8_t* out, int64_t i, float y) {
@@ -402,7 +424,7 @@ __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c
                 Ls += f * __ldcg(pl + s2 * G + h);
                 O += f * __ldcg(p.ws_o + (int64_t(bg + c0 + s2) * G + h) * D + c);
             }
-            write_out<T>(p.out, out_row0 * D + idx, Ls > 0.f ? O / Ls : 0.f);
+            emit<T, D>(p, out_row0 + h, c, M, Ls, O);
         }
         return true;
     }
@@ -438,12 +460,20 @@ __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c
             O.x += f * o.x; O.y += f * o.y; O.z += f * o.z; O.w += f * o.w;
         }
         const float Ls = Mh[G + h];
-        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-        const int64_t o0 = out_row0 * D + int64_t(q4) * 4;
-        write_out<T>(p.out, o0 + 0, O.x * inv);
-        write_out<T>(p.out, o0 + 1, O.y * inv);
-        write_out<T>(p.out, o0 + 2, O.z * inv);
-        write_out<T>(p.out, o0 + 3, O.w * inv);
+        const int c = (q4 * 4) % D;
+        if (p.part_out != nullptr) {
+            emit<T, D>(p, out_row0 + h, c + 0, Mh[h], Ls, O.x);
+            emit<T, D>(p, out_row0 + h, c + 1, Mh[h], Ls, O.y);
+            emit<T, D>(p, out_row0 + h, c + 2, Mh[h], Ls, O.z);
+            emit<T, D>(p, out_row0 + h, c + 3, Mh[h], Ls, O.w);
+        } else {
+            const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+            const int64_t o0 = out_row0 * D + int64_t(q4) * 4;
+            write_out<T>(p.out, o0 + 0, O.x * inv);
+            write_out<T>(p.out, o0 + 1, O.y * inv);
+            write_out<T>(p.out, o0 + 2, O.z * inv);
+            write_out<T>(p.out, o0 + 3, O.w * inv);
+        }
     }
     return ok;
 }
@@ -492,9 +522,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     // sequences with no cached positions: zero output (CTA b mod grid writes it)
     for (int b = blockIdx.x; b < p.batch; b += p.num_ctas) {
         if (s_ts[b + 1] != s_ts[b]) continue;
-        for (int idx = tid; idx < p.hq * D; idx += blockDim.x) {
-            write_out<T>(p.out, int64_t(b) * p.hq * D + idx, 0.f);
-        }
+        for (int idx = tid; idx < p.hq * D; idx += blockDim.x)
+            emit<T, D>(p, int64_t(b) * p.hq + idx / D, idx % D, NEG_INF_F, 0.f, 0.f);
     }
 
     const int total = s_ts[p.batch];
@@ -684,7 +713,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                     }
                 }
                 if (whole) {
-                    write_out<T>(p.out, (int64_t(mt.b) * p.hq + mt.g * G + h) * D + c, Ls > 0.f ? O / Ls : 0.f);
+                    emit<T, D>(p, int64_t(mt.b) * p.hq + mt.g * G + h, c, M, Ls, O);
                 } else {
                     p.ws_o[(int64_t(slot) * G + h) * D + c] = O;
                     if (c == 0) {
@@ -733,6 +762,29 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
     __syncwarp();
     if (lane == 0) atomicAdd(&s_cdone, 1);
+}
+
+// Merge R unnormalised partials [R][rows][D + 2] (o, m, l per row, as the
+// partial mode writes them) into out [rows][D]: M = max_r m_r,
+// out = sum_r 2^{m_r - M} o_r / sum_r 2^{m_r - M} l_r; rows with no tokens
+// anywhere (all m = -inf) give 0.  One CTA per row, one thread per channel.
+template <typename T, int D>
+__global__ void __launch_bounds__(D) combine_parts_kernel(const float* parts, int nparts, int64_t rows, uint8_t* out) {
+    const int64_t row = blockIdx.x;
+    const int c = threadIdx.x;
+    const int64_t stride = rows * (D + 2);
+    float M = NEG_INF_F;
+    for (int r = 0; r < nparts; ++r) M = fmaxf(M, parts[r * stride + row * (D + 2) + D]);
+    float Ls = 0.f, O = 0.f;
+    if (M != NEG_INF_F) {
+        for (int r = 0; r < nparts; ++r) {
+            const float* pr = parts + r * stride + row * (D + 2);
+            const float f = exp2f(pr[D] - M);
+            Ls += f * pr[D + 1];
+            O += f * pr[c];
+        }
+    }
+    write_out<T>(out, row * D + c, Ls > 0.f ? O / Ls : 0.f);
 }
 
 }  // namespace yocopp

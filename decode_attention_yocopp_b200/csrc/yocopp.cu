@@ -335,14 +335,14 @@ int64_t yocopp_decode_attn_workspace_size(const yocopp_cache* cache, int32_t num
                                     sms * YOCOPP_DECODE_CTAS_PER_SM).total);
 }
 
-int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32_t* seq_lens, void* out,
-                           int32_t num_q_heads, float scale, void* workspace, int64_t workspace_bytes,
-                           void* stream) {
+static int32_t decode_attn_impl(const void* q, const yocopp_cache* cache, const int32_t* seq_lens, void* out,
+                                float* part_out, int32_t num_q_heads, float scale, void* workspace,
+                                int64_t workspace_bytes, void* stream) {
     int G = 0;
     int32_t rc = check_decode_shape(cache, num_q_heads, &G);
     if (rc != YOCOPP_OK) return rc;
-    if (q == nullptr || out == nullptr || seq_lens == nullptr) return YOCOPP_EINVAL;
-    if (!aligned(q, 16) || !aligned(out, 16)) return YOCOPP_EINVAL;
+    if (q == nullptr || (out == nullptr && part_out == nullptr) || seq_lens == nullptr) return YOCOPP_EINVAL;
+    if (!aligned(q, 16) || !aligned(out != nullptr ? out : static_cast<void*>(part_out), 16)) return YOCOPP_EINVAL;
     if (!(scale >= 0.f) || !std::isfinite(scale)) return YOCOPP_EINVAL;
     const int sms = sm_count(current_device());
     if (sms <= 0) return YOCOPP_ECUDA;
@@ -386,6 +386,7 @@ int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32
     p.drop_tile = g_test_drop_tile;
     p.wait_limit_ns = g_wait_limit_ns;
     p.epoch = next_epoch();
+    p.part_out = part_out;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
 #define YOCOPP_DECODE_CASE(TT, DD)                                             \
@@ -401,6 +402,41 @@ int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32
     if (D == 128) { YOCOPP_DECODE_CASE(float, 128) }
     YOCOPP_DECODE_CASE(float, 64)
 #undef YOCOPP_DECODE_CASE
+}
+
+int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32_t* seq_lens, void* out,
+                           int32_t num_q_heads, float scale, void* workspace, int64_t workspace_bytes,
+                           void* stream) {
+    if (out == nullptr) return YOCOPP_EINVAL;
+    return decode_attn_impl(q, cache, seq_lens, out, nullptr, num_q_heads, scale, workspace, workspace_bytes,
+                            stream);
+}
+
+int32_t yocopp_decode_attn_partial(const void* q, const yocopp_cache* cache, const int32_t* seq_lens,
+                                   float* partial, int32_t num_q_heads, float scale, void* workspace,
+                                   int64_t workspace_bytes, void* stream) {
+    if (partial == nullptr) return YOCOPP_EINVAL;
+    return decode_attn_impl(q, cache, seq_lens, nullptr, partial, num_q_heads, scale, workspace,
+                            workspace_bytes, stream);
+}
+
+int32_t yocopp_decode_combine(const float* partials, int32_t num_parts, int64_t rows, int32_t head_dim,
+                              int32_t dtype, void* out, void* stream) {
+    if (partials == nullptr || out == nullptr || num_parts < 1 || rows < 0) return YOCOPP_EINVAL;
+    if (elem_bytes(dtype) == 0) return YOCOPP_EDTYPE;
+    if (head_dim != 64 && head_dim != 128) return YOCOPP_EINVAL;
+    if (rows == 0) return YOCOPP_OK;
+    if (rows > (int64_t(1) << 31) - 1) return YOCOPP_EINVAL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* o = static_cast<uint8_t*>(out);
+    if (dtype == YOCOPP_BF16) {
+        if (head_dim == 128) combine_parts_kernel<__nv_bfloat16, 128><<<unsigned(rows), 128, 0, st>>>(partials, num_parts, rows, o);
+        else combine_parts_kernel<__nv_bfloat16, 64><<<unsigned(rows), 64, 0, st>>>(partials, num_parts, rows, o);
+    } else {
+        if (head_dim == 128) combine_parts_kernel<float, 128><<<unsigned(rows), 128, 0, st>>>(partials, num_parts, rows, o);
+        else combine_parts_kernel<float, 64><<<unsigned(rows), 64, 0, st>>>(partials, num_parts, rows, o);
+    }
+    return cuda_status(cudaGetLastError());
 }
 
 // Decode attention whose workspace is the library's own static device array

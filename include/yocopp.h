@@ -165,6 +165,34 @@ int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32
                            int64_t workspace_bytes, void* stream);
 
 /*
+ * yocopp_decode_attn_partial - yocopp_decode_attn over this caller's cached
+ * positions only, kept unnormalised so that it can be merged with results
+ * over other positions of the same sequences (for example other GPUs' shards
+ * of one long context; You Only Cache Once, abstract: the cache scales to
+ * 1M tokens, more than one GPU holds).  Arguments as yocopp_decode_attn,
+ * with `partial` in place of `out`:
+ *   partial : device fp32 [batch][num_q_heads][head_dim + 2]; per row the
+ *             weighted sum o[c] = sum_t 2^(s'_t - m) V'_t[c] for c < head_dim,
+ *             then m = max_t s'_t and l = sum_t 2^(s'_t - m), where
+ *             s'_t = scale * log2(e) * <q, K'_t> (base-2 logits).  A sequence
+ *             with no positions gives o = 0, m = -inf, l = 0.
+ */
+int32_t yocopp_decode_attn_partial(const void* q, const yocopp_cache* cache, const int32_t* seq_lens,
+                                   float* partial, int32_t num_q_heads, float scale, void* workspace,
+                                   int64_t workspace_bytes, void* stream);
+
+/*
+ * yocopp_decode_combine - exact log-sum-exp merge of num_parts partial results
+ * (each laid out as yocopp_decode_attn_partial writes them) into the output:
+ *   partials : device fp32 [num_parts][rows][head_dim + 2], rows = batch * num_q_heads
+ *   out      : device [rows][head_dim] of `dtype`
+ * out = sum_r 2^(m_r - M) o_r / sum_r 2^(m_r - M) l_r with M = max_r m_r;
+ * rows with no positions in any part give 0.
+ */
+int32_t yocopp_decode_combine(const float* partials, int32_t num_parts, int64_t rows, int32_t head_dim,
+                              int32_t dtype, void* out, void* stream);
+
+/*
  * yocopp_decode_attn_static - yocopp_decode_attn without a caller workspace.
  * The paper has no counterpart: this entry point exists for callers that
  * cannot allocate device memory on this path, such as a host framework that

@@ -70,3 +70,17 @@ def decode_group(orc: Oracle, w: "gen.Workload", layer: int, b: int, g: int,
         K, V = kv
     q = query(w, layer, b)[g * w.group:(g + 1) * w.group]
     return orc.attention(q, K, V, w.dtype, default_scale(w.d) if scale is None else scale)
+
+
+def decode_self_group(orc: Oracle, w: "gen.Workload", layer: int, b: int, g: int,
+                      kv: Tuple[np.ndarray, np.ndarray] | None = None, scale: float | None = None) -> np.ndarray:
+    """Self-decoder layer ``layer`` (1..L/2) attending over its own stored cache during
+    decode (YOCO++ section 2, cache strategy: each lower-half layer reads the one KV set
+    it stored): [G][d] fp64 for the query heads of KV head g, q from that layer."""
+    if kv is None:
+        K = composed_seq(orc, w, layer, "K", b, g)
+        V = composed_seq(orc, w, layer, "V", b, g)
+    else:
+        K, V = kv
+    q = query(w, layer, b)[g * w.group:(g + 1) * w.group]
+    return orc.attention(q, K, V, w.dtype, default_scale(w.d) if scale is None else scale)

@@ -108,3 +108,22 @@ def test_planted_literal_reading(orc):
     outs = decode_layers(w, stack, lens, layers=w.cross_layers[:3])
     for g in range(w.hkv):
         _check_plane(orc, w, stack, outs, 0, g, w.cross_layers[:3])
+
+
+def test_self_decoder_layers(orc):
+    """Self-decoder decode attention: every lower-half layer (raw layer 1 and the
+    composed layers 2..L/2) attends over its own cache with its own query."""
+    w = gen.config(2, lens=[1000, 3000, 1, 64])
+    layers = [1, 2, 7, w.shared_layer]
+    stack = device_stack(w, compose_layers=layers)
+    lens = write_layers(w, stack, layers)
+    tdt = torch.bfloat16
+    for i in layers:
+        q = w.device(gen.Q, i)
+        out = torch.empty((w.batch, w.hq, w.d), dtype=tdt, device="cuda")
+        stack.self_attend(i, q, lens, out)
+        got_all = np_storage(out)
+        for b in range(w.batch):
+            for g in (0, w.hkv - 1):
+                ref = model.decode_self_group(orc, w, i, b, g)
+                assert_attention(got_all[b, g * w.group:(g + 1) * w.group], ref, w.dtype, orc, f"self layer {i} b{b} g{g}")
