@@ -242,6 +242,35 @@ class Step:
         self.prefill_ntok = w.total_prefill
         self.launches_per_step = 2 * len(comp) + len(self.cross)  # compose x2 per layer, one decode launch per layer
 
+    def setup_fused_contrast(self):
+        """Raw caches for the read-time composition contrast: layer 1 (already raw) and a raw
+        copy of the shared layer, written at the init alpha (which stores the inputs as they are)."""
+        import torch
+        from decode_attention_yocopp_b200 import alloc_workspace, make_cache, yocopp_compose_append
+        w = self.w
+        L2 = w.shared_layer
+        k = torch.empty_like(self.stack.k[L2])
+        v = torch.empty_like(self.stack.v[L2])
+        self.raw_shared = make_cache(k, v, self.bt if w.paged else None)
+        init = (0.0, 1.0 / w.lam, 0.0, 1.0 / w.lam)
+        if self.cu is None:
+            yocopp_compose_append(self.kp[L2], self.vp[L2], self.kp[L2], self.vp[L2], init, w.lam, self.raw_shared,
+                                  self.pos0, n_uniform=w.lens[0] - 1, total_new=self.kp[L2].shape[0])
+        else:
+            yocopp_compose_append(self.kp[L2], self.vp[L2], self.kp[L2], self.vp[L2], init, w.lam, self.raw_shared,
+                                  self.pos0, cu_new=self.cu, total_new=self.kp[L2].shape[0])
+        yocopp_compose_append(self.kn[L2], self.vn[L2], self.kn[L2], self.vn[L2], init, w.lam, self.raw_shared,
+                              self.posn, n_uniform=1, total_new=w.batch)
+        self.fused_ws = alloc_workspace(self.raw_shared, w.hq)
+
+    def run_fused(self):
+        """Every cross-decoder layer with K', V' composed at read time from two raw caches."""
+        from decode_attention_yocopp_b200 import yocopp_decode_attn_fused
+        w = self.w
+        for l in self.cross:
+            yocopp_decode_attn_fused(self.q[l], self.raw_shared, self.stack.desc[1], w.alpha[w.shared_layer], w.lam,
+                                     self.lens, self.out[l], self.fused_ws)
+
     def write_layer1_prefill(self):
         """Layer 1 stores its raw K_1, V_1 (set up once; the composed layers are written every step)."""
         w, s = self.w, self.stack
@@ -364,6 +393,20 @@ def run_ours(args, rank, world, local):
     t_self_max = max_over_ranks(t_self, world)
     self_bytes = sum_over_ranks(w.kv_bytes() * len(step.selfl) * K, world)
 
+    # contrast: the same cross-decoder layers composing K', V' at read time (2x the bytes)
+    step.setup_fused_contrast()
+    for _ in range(2):
+        step.run_fused()
+    torch.cuda.synchronize()
+    barrier(world)
+    fa = _event()
+    for _ in range(K):
+        step.run_fused()
+    fb = _event()
+    torch.cuda.synchronize()
+    t_fused_max = max_over_ranks(fa.elapsed_time(fb), world)
+    del step.raw_shared, step.fused_ws
+
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, step, world)
@@ -412,6 +455,12 @@ def run_ours(args, rank, world, local):
                              "self_attn_kv_gbs": round(self_bytes / (t_self_max * 1e-3) / 1e9, 1),
                              "what": "decoded token appended to layers 1..L/2, L/2 self-decoder attentions over "
                                      "their own caches, L/2 cross-decoder attentions over the shared cache"},
+        "read_time_composition_contrast": {
+            "what": "cross-decoder attention composing K', V' from two raw caches while decoding "
+                    "(the FusedKV-style alternative); YOCO++ reads one composed cache instead",
+            "ms_per_step": round(t_fused_max / K, 4),
+            "hbm_read_gbs": round(2 * kv_all / (t_fused_max * 1e-3) / 1e9, 1),
+            "slowdown_vs_composed_cache": round(t_fused_max / t_attn_max, 3)},
         "roofline": dominant,
         "profiling_trim": bool(args.compose_layers or args.cross_layers),
         "roofline_attention": roof_attn,

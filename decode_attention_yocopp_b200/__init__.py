@@ -30,7 +30,7 @@ YOCOPP_F32 = 1
 EXPORTS = ("yocopp_compose_append", "yocopp_decode_attn_workspace_size", "yocopp_decode_attn",
            "yocopp_get_device_status", "yocopp_status_string", "yocopp_version",
            "yocopp_testing_set_decode_fault", "yocopp_decode_attn_static", "yocopp_decode_attn_partial",
-           "yocopp_decode_combine")
+           "yocopp_decode_combine", "yocopp_decode_attn_fused")
 
 
 class yocopp_cache(ctypes.Structure):
@@ -76,6 +76,10 @@ def load(path: Optional[str] = None):
     lib.yocopp_testing_set_decode_fault.argtypes = [I32, I64]
     lib.yocopp_decode_attn_partial.restype = I32
     lib.yocopp_decode_attn_partial.argtypes = [V, ctypes.POINTER(yocopp_cache), V, V, I32, ctypes.c_float, V, I64, V]
+    lib.yocopp_decode_attn_fused.restype = I32
+    lib.yocopp_decode_attn_fused.argtypes = [V, ctypes.POINTER(yocopp_cache), ctypes.POINTER(yocopp_cache),
+                                             ctypes.POINTER(ctypes.c_float), ctypes.c_float, V, V, I32,
+                                             ctypes.c_float, V, I64, V]
     lib.yocopp_decode_combine.restype = I32
     lib.yocopp_decode_combine.argtypes = [V, I32, I64, I32, I32, V, V]
     lib.yocopp_decode_attn_static.restype = I32
@@ -187,6 +191,19 @@ def yocopp_decode_attn_partial(q, cache: yocopp_cache, seq_lens, partial, worksp
                                            workspace.numel() * workspace.element_size() if workspace is not None else 0,
                                            _stream(stream))
     _check("yocopp_decode_attn_partial", rc)
+
+
+def yocopp_decode_attn_fused(q, cache_i: yocopp_cache, cache_1: yocopp_cache, alpha: Sequence[float], lam: float,
+                             seq_lens, out, workspace, num_q_heads: Optional[int] = None, scale: float = 0.0,
+                             stream=None) -> None:
+    """Decode attention composing K', V' at read time from two raw caches (twice the bytes)."""
+    hq = q.shape[1] if num_q_heads is None else num_q_heads
+    a = (ctypes.c_float * 4)(*[float(x) for x in alpha])
+    rc = load().yocopp_decode_attn_fused(_ptr(q), ctypes.byref(cache_i), ctypes.byref(cache_1), a, float(lam),
+                                         _ptr(seq_lens), _ptr(out), int(hq), float(scale), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size() if workspace is not None else 0,
+                                         _stream(stream))
+    _check("yocopp_decode_attn_fused", rc)
 
 
 def yocopp_decode_combine(partials, out, stream=None) -> None:

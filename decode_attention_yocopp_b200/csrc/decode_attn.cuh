@@ -50,6 +50,7 @@ struct DecodeParams {
     uint64_t wait_limit_ns;
     unsigned long long epoch;    // grows with every call (44 bits, never 0): tags this call's arrivals
     float* part_out;             // non-null: write unnormalised [batch][hq][D + 2] (o, m, l) instead of out
+    float fa1k, fa2k, fa1v, fa2v;  // read-time composition (fused variant): lambda * alpha
 };
 
 struct TileMeta {
@@ -57,15 +58,18 @@ struct TileMeta {
 };
 enum : int32_t { kFirst = 1, kLast = 2, kWhole = 4 };
 
-template <int D, typename T>
+// FUSED: the stage also holds the layer-1 K/V tiles and K'/V' are composed at
+// read time (twice the bytes per token, so the tile is halved).
+template <int D, typename T, bool FUSED = false>
 struct DecodeShape {
     static constexpr int EB = sizeof(T);
     static constexpr int ROWB = D * EB;                   // bytes per (token, head) row
-    static constexpr int TILE = ROWB <= 256 ? 64 : 32;    // tokens per pipeline tile
+    static constexpr int TILE = (ROWB <= 256 ? 64 : 32) / (FUSED ? 2 : 1);  // tokens per pipeline tile
     static constexpr int NBOX = ROWB / 128;               // 128-byte swizzle boxes per row
     static constexpr int BOXB = TILE * 128;               // bytes of one box column of a tile
     static constexpr int KV_BYTES = TILE * ROWB;          // one K (or V) tile
-    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+    static constexpr int NSRC = FUSED ? 4 : 2;            // tiles per stage: K, V (, K_1, V_1)
+    static constexpr int STAGE_BYTES = NSRC * KV_BYTES;
     static constexpr int CPR = ROWB / 16;                 // 16-byte chunks per row
     static constexpr int CPL = CPR / 8;                   // score phase: chunks per lane
     static constexpr int EPC = 16 / EB;                   // elements per chunk
@@ -149,9 +153,9 @@ __device__ void tile_prefix(const DecodeParams& p, int* s_ts, int* s_warp) {
     __syncthreads();
 }
 
-template <typename T, int D, int G, int W, int STAGES>
+template <typename T, int D, int G, int W, int STAGES, bool FUSED = false>
 struct DecodeSmem {
-    using S = DecodeShape<D, T>;
+    using S = DecodeShape<D, T, FUSED>;
     static constexpr int TPW = S::TILE / W;
     static constexpr size_t up16(size_t x) { return (x + 15) & ~size_t(15); }
     static constexpr size_t kStages = size_t(STAGES) * S::STAGE_BYTES;      // 1024-aligned ring
@@ -181,9 +185,38 @@ __device__ __forceinline__ unsigned arrive_plane(unsigned long long* cnt, unsign
 // Per-warp state and work of a consumer warp: the group's queries in
 // registers, the online-softmax running maxima / partial sums, and the
 // running weighted value sums for this warp's share of every tile.
-template <typename T, int D, int G, int W>
+// One 16-byte chunk of a K or V tile as EPC/2 fp32 pairs; with FUSED, composed
+// at read time from the layer-L/2 and layer-1 tiles: (lambda a2) xi + (lambda a1) x1.
+template <typename T, bool FUSED, int NP>
+__device__ __forceinline__ void load_pairs(const uint8_t* a, const uint8_t* a1, float2 c1, float2 c2,
+                                           float2 (&out)[NP]) {
+    const uint4 v = *reinterpret_cast<const uint4*>(a);
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) out[e] = bf16x2_to_float2(w[e]);
+    } else {
+        out[0] = make_float2(__uint_as_float(w[0]), __uint_as_float(w[1]));
+        out[1] = make_float2(__uint_as_float(w[2]), __uint_as_float(w[3]));
+    }
+    if constexpr (FUSED) {
+        const uint4 v1 = *reinterpret_cast<const uint4*>(a1);
+        const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&v1);
+#pragma unroll
+        for (int e = 0; e < NP; ++e) {
+            float2 x1;
+            if constexpr (sizeof(T) == 2)
+                x1 = bf16x2_to_float2(w1[e]);
+            else
+                x1 = make_float2(__uint_as_float(w1[2 * e]), __uint_as_float(w1[2 * e + 1]));
+            out[e] = ffma2(c1, x1, fmul2(c2, out[e]));
+        }
+    }
+}
+
+template <typename T, int D, int G, int W, bool FUSED = false>
 struct ConsumerWarp {
-    using S = DecodeShape<D, T>;
+    using S = DecodeShape<D, T, FUSED>;
     static constexpr int TILE = S::TILE, TPW = TILE / W, CPR = S::CPR, CPL = S::CPL, EPC = S::EPC, TPI = S::TPI;
     static constexpr int QK_IT = TPW / 4;     // score steps (4 tokens per step)
     static constexpr int PV_IT = TPW / TPI;   // value steps (TPI tokens per step)
@@ -230,31 +263,22 @@ struct ConsumerWarp {
         m_mine = NEG_INF_F;
     }
 
+    float2 fk1, fk2, fv1, fv2;    // read-time composition coefficients (fused variant)
+
     // Score of one token row for head hr (8 lanes per token, packed FMAs, reduce-scatter).
-    __device__ __forceinline__ float score(const uint8_t* Kt, int row) const {
+    __device__ __forceinline__ float score(const uint8_t* Kt, const uint8_t* K1t, int row) const {
         float2 part[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) part[h] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int jb = 0; jb < CPL; ++jb) {
-            const uint4 kv = *reinterpret_cast<const uint4*>(Kt + jb * S::BOXB + row * 128 + ((r8 ^ (row & 7)) << 4));
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(&kv);
-            if constexpr (S::EB == 2) {
+            const int off = jb * S::BOXB + row * 128 + ((r8 ^ (row & 7)) << 4);
+            float2 kf[EPC / 2];
+            load_pairs<T, FUSED>(Kt + off, K1t + off, fk1, fk2, kf);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 kf = bf16x2_to_float2(w[e]);
+            for (int e = 0; e < EPC / 2; ++e)
 #pragma unroll
-                    for (int h = 0; h < G; ++h) part[h] = ffma2(q2[h][jb * 4 + e], kf, part[h]);
-                }
-            } else {
-                const float2 k0 = make_float2(__uint_as_float(w[0]), __uint_as_float(w[1]));
-                const float2 k1 = make_float2(__uint_as_float(w[2]), __uint_as_float(w[3]));
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    part[h] = ffma2(q2[h][jb * 2 + 0], k0, part[h]);
-                    part[h] = ffma2(q2[h][jb * 2 + 1], k1, part[h]);
-                }
-            }
+                for (int h = 0; h < G; ++h) part[h] = ffma2(q2[h][jb * (EPC / 2) + e], kf[e], part[h]);
         }
         float v[G];
 #pragma unroll
@@ -290,10 +314,12 @@ struct ConsumerWarp {
     template <bool MASK>
     __device__ __forceinline__ void tile(const uint8_t* Kt, const uint8_t* Vt, float2* p2, int tok0, int len) {
         const int rbase = warp * TPW;
+        const uint8_t* K1t = Kt + 2 * S::KV_BYTES;  // layer-1 tiles (fused variant only)
+        const uint8_t* V1t = Kt + 3 * S::KV_BYTES;
         float s[QK_IT];
 #pragma unroll
         for (int i = 0; i < QK_IT; ++i) {
-            s[i] = score(Kt, rbase + i * 4 + j4);
+            s[i] = score(Kt, K1t, rbase + i * 4 + j4);
             if (MASK && tok0 + i * 4 + j4 >= len) s[i] = NEG_INF_F;
         }
         // maxima of this slice per head, then the (warp-uniform) running update
@@ -336,8 +362,13 @@ struct ConsumerWarp {
         for (int i2 = 0; i2 < PV_IT; ++i2) {
             const int tl = i2 * TPI + pslot;  // token within the slice
             const int tk = rbase + tl;        // row within the tile
-            uint4 vv = *reinterpret_cast<const uint4*>(Vt + pbx * S::BOXB + tk * 128 + ((pcc ^ (tk & 7)) << 4));
-            if (MASK && tok0 + tl >= len) vv = make_uint4(0u, 0u, 0u, 0u);  // never use rows past the sequence
+            const int voff = pbx * S::BOXB + tk * 128 + ((pcc ^ (tk & 7)) << 4);
+            float2 vf[EPC / 2];
+            load_pairs<T, FUSED>(Vt + voff, V1t + voff, fv1, fv2, vf);
+            if (MASK && tok0 + tl >= len) {  // never use rows past the sequence
+#pragma unroll
+                for (int e = 0; e < EPC / 2; ++e) vf[e] = make_float2(0.f, 0.f);
+            }
             float2 pp[G];
             if constexpr (G >= 2) {
 #pragma unroll
@@ -348,15 +379,6 @@ struct ConsumerWarp {
                 }
             } else {
                 pp[0] = p2[tl];
-            }
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(&vv);
-            float2 vf[EPC / 2];
-            if constexpr (S::EB == 2) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) vf[e] = bf16x2_to_float2(w[e]);
-            } else {
-                vf[0] = make_float2(__uint_as_float(w[0]), __uint_as_float(w[1]));
-                vf[1] = make_float2(__uint_as_float(w[2]), __uint_as_float(w[3]));
             }
 #pragma unroll
             for (int h = 0; h < G; ++h)
@@ -478,12 +500,13 @@ __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c
     return ok;
 }
 
-template <typename T, int D, int G, int W, int STAGES, int CTAS_PER_SM>
+template <typename T, int D, int G, int W, int STAGES, int CTAS_PER_SM, bool FUSED>
 __global__ void __launch_bounds__((W + 1) * 32, CTAS_PER_SM)
 decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmV1,
                     const DecodeParams p) {
-    using S = DecodeShape<D, T>;
-    using L = DecodeSmem<T, D, G, W, STAGES>;
+    using S = DecodeShape<D, T, FUSED>;
+    using L = DecodeSmem<T, D, G, W, STAGES, FUSED>;
     constexpr int TILE = S::TILE, TPW = L::TPW;
 
     extern __shared__ uint8_t smem_raw[];
@@ -537,6 +560,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         if (lane == 0) {
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
+            if constexpr (FUSED) {
+                prefetch_tensormap(&tmK1);
+                prefetch_tensormap(&tmV1);
+            }
         }
         constexpr int NSB_MAX = 4;  // sub-boxes per tile when blocks are shorter than a tile
         const int nsb = TILE / p.boxr;
@@ -615,7 +642,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                     if (start + it != p.drop_tile) {
                         uint32_t nvalid = 0;
                         for (int s = 0; s < nsb; ++s) nvalid += r[s] >= 0 ? 1u : 0u;
-                        const uint32_t bytes = nvalid * uint32_t(S::NBOX * p.boxr * 128 * 2);
+                        const uint32_t bytes = nvalid * uint32_t(S::NBOX * p.boxr * 128 * S::NSRC);
                         mbar_arrive_expect_tx(&full_bar[stage], bytes);
                         uint8_t* kdst = stage_mem + size_t(stage) * S::STAGE_BYTES;
                         uint8_t* vdst = kdst + S::KV_BYTES;
@@ -626,6 +653,12 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                                 const int off = bx * S::BOXB + s * p.boxr * 128;
                                 tma_load_2d(kdst + off, &tmK, &full_bar[stage], bx * (128 / S::EB), r[s]);
                                 tma_load_2d(vdst + off, &tmV, &full_bar[stage], bx * (128 / S::EB), r[s]);
+                                if constexpr (FUSED) {
+                                    tma_load_2d(kdst + 2 * S::KV_BYTES + off, &tmK1, &full_bar[stage],
+                                                bx * (128 / S::EB), r[s]);
+                                    tma_load_2d(kdst + 3 * S::KV_BYTES + off, &tmV1, &full_bar[stage],
+                                                bx * (128 / S::EB), r[s]);
+                                }
                             }
                         }
                         last_issued_it[stage] = it;
@@ -650,7 +683,11 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
 
     // ---------------------------------------------------------------------- consumers
-    ConsumerWarp<T, D, G, W> cw(warp, lane);
+    ConsumerWarp<T, D, G, W, FUSED> cw(warp, lane);
+    cw.fk1 = make_float2(p.fa1k, p.fa1k);
+    cw.fk2 = make_float2(p.fa2k, p.fa2k);
+    cw.fv1 = make_float2(p.fa1v, p.fa1v);
+    cw.fv2 = make_float2(p.fa2v, p.fa2v);
     __shared__ int s_last;
     float2* p2 = reinterpret_cast<float2*>(p_s) + warp * TPW * G;  // this warp's (p, p) pairs
 

@@ -138,18 +138,19 @@ struct DecodeLaunch {
     int w, stages, tile, ctas_per_sm;
 };
 
-template <typename T, int D>
+template <typename T, int D, bool FUSED>
 constexpr DecodeLaunch decode_cfg() {
-    return DecodeLaunch{YOCOPP_DECODE_WARPS, YOCOPP_DECODE_STAGES, DecodeShape<D, T>::TILE,
+    return DecodeLaunch{YOCOPP_DECODE_WARPS, YOCOPP_DECODE_STAGES, DecodeShape<D, T, FUSED>::TILE,
                         YOCOPP_DECODE_CTAS_PER_SM};
 }
 
-template <typename T, int D, int G>
-int32_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, cudaStream_t st) {
-    constexpr DecodeLaunch cfg = decode_cfg<T, D>();
+template <typename T, int D, int G, bool FUSED>
+int32_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tk1, const CUtensorMap& tv1,
+                      const DecodeParams& p, cudaStream_t st) {
+    constexpr DecodeLaunch cfg = decode_cfg<T, D, FUSED>();
     constexpr int W = cfg.w, STAGES = cfg.stages;
-    auto kern = decode_split_kernel<T, D, G, W, STAGES, cfg.ctas_per_sm>;
-    const size_t smem = DecodeSmem<T, D, G, W, STAGES>::bytes(p.batch);
+    auto kern = decode_split_kernel<T, D, G, W, STAGES, cfg.ctas_per_sm, FUSED>;
+    const size_t smem = DecodeSmem<T, D, G, W, STAGES, FUSED>::bytes(p.batch);
     static bool attr_set[kMaxDevices] = {false};
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices) return YOCOPP_ECUDA;
@@ -178,7 +179,7 @@ int32_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const Decode
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
     lc.numAttrs = 1;
-    return cuda_status(cudaLaunchKernelEx(&lc, kern, tk, tv, p));
+    return cuda_status(cudaLaunchKernelEx(&lc, kern, tk, tv, tk1, tv1, p));
 }
 
 struct WorkspaceLayout {
@@ -335,12 +336,31 @@ int64_t yocopp_decode_attn_workspace_size(const yocopp_cache* cache, int32_t num
                                     sms * YOCOPP_DECODE_CTAS_PER_SM).total);
 }
 
+// fused != nullptr: the read-time composition variant; `cache` holds raw K_i, V_i,
+// fused->cache1 raw K_1, V_1 (same shape and layout), fused->coef = lambda * alpha.
+struct FusedArgs {
+    const yocopp_cache* cache1;
+    float coef[4];
+};
+
 static int32_t decode_attn_impl(const void* q, const yocopp_cache* cache, const int32_t* seq_lens, void* out,
                                 float* part_out, int32_t num_q_heads, float scale, void* workspace,
-                                int64_t workspace_bytes, void* stream) {
+                                int64_t workspace_bytes, void* stream, const FusedArgs* fused = nullptr) {
     int G = 0;
     int32_t rc = check_decode_shape(cache, num_q_heads, &G);
     if (rc != YOCOPP_OK) return rc;
+    if (fused != nullptr) {
+        const yocopp_cache* c1 = fused->cache1;
+        rc = check_cache(c1);
+        if (rc != YOCOPP_OK) return rc;
+        if (c1->dtype != cache->dtype || c1->batch != cache->batch || c1->num_kv_heads != cache->num_kv_heads ||
+            c1->head_dim != cache->head_dim || c1->capacity != cache->capacity ||
+            c1->block_table != cache->block_table ||
+            (cache->block_table != nullptr && (c1->block_size != cache->block_size ||
+                                               c1->max_blocks_per_seq != cache->max_blocks_per_seq ||
+                                               c1->num_blocks != cache->num_blocks)))
+            return YOCOPP_EINVAL;
+    }
     if (q == nullptr || (out == nullptr && part_out == nullptr) || seq_lens == nullptr) return YOCOPP_EINVAL;
     if (!aligned(q, 16) || !aligned(out != nullptr ? out : static_cast<void*>(part_out), 16)) return YOCOPP_EINVAL;
     if (!(scale >= 0.f) || !std::isfinite(scale)) return YOCOPP_EINVAL;
@@ -352,15 +372,23 @@ static int32_t decode_attn_impl(const void* q, const yocopp_cache* cache, const 
         return YOCOPP_EWORKSPACE;
 
     const int D = cache->head_dim;
-    const int tile = (D * elem_bytes(cache->dtype)) <= 256 ? 64 : 32;
+    const int tile = ((D * elem_bytes(cache->dtype)) <= 256 ? 64 : 32) / (fused != nullptr ? 2 : 1);
     const bool paged = cache->block_table != nullptr;
     const int boxr = paged ? (cache->block_size < tile ? cache->block_size : tile) : tile;
     const int64_t rows = paged ? int64_t(cache->num_blocks) * cache->num_kv_heads * cache->block_size
                                : int64_t(cache->batch) * cache->num_kv_heads * cache->capacity;
-    alignas(64) CUtensorMap tk, tv;
+    alignas(64) CUtensorMap tk, tv, tk1, tv1;
     if (!encode_rows(&tk, cache->k, cache->dtype, D, rows, boxr) ||
         !encode_rows(&tv, cache->v, cache->dtype, D, rows, boxr))
         return YOCOPP_ECUDA;
+    if (fused != nullptr) {
+        if (!encode_rows(&tk1, fused->cache1->k, cache->dtype, D, rows, boxr) ||
+            !encode_rows(&tv1, fused->cache1->v, cache->dtype, D, rows, boxr))
+            return YOCOPP_ECUDA;
+    } else {
+        tk1 = tk;
+        tv1 = tv;
+    }
 
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     DecodeParams p;
@@ -387,20 +415,32 @@ static int32_t decode_attn_impl(const void* q, const yocopp_cache* cache, const 
     p.wait_limit_ns = g_wait_limit_ns;
     p.epoch = next_epoch();
     p.part_out = part_out;
+    p.fa1k = fused ? fused->coef[0] : 0.f;
+    p.fa2k = fused ? fused->coef[1] : 0.f;
+    p.fa1v = fused ? fused->coef[2] : 0.f;
+    p.fa2v = fused ? fused->coef[3] : 0.f;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-#define YOCOPP_DECODE_CASE(TT, DD)                                             \
-    switch (G) {                                                               \
-        case 1: return launch_decode<TT, DD, 1>(tk, tv, p, st);                \
-        case 2: return launch_decode<TT, DD, 2>(tk, tv, p, st);                \
-        default: return launch_decode<TT, DD, 4>(tk, tv, p, st);               \
+#define YOCOPP_DECODE_CASE(TT, DD, FF)                                                 \
+    switch (G) {                                                                       \
+        case 1: return launch_decode<TT, DD, 1, FF>(tk, tv, tk1, tv1, p, st);          \
+        case 2: return launch_decode<TT, DD, 2, FF>(tk, tv, tk1, tv1, p, st);          \
+        default: return launch_decode<TT, DD, 4, FF>(tk, tv, tk1, tv1, p, st);         \
+    }
+    if (fused != nullptr) {
+        if (cache->dtype == YOCOPP_BF16) {
+            if (D == 128) { YOCOPP_DECODE_CASE(__nv_bfloat16, 128, true) }
+            YOCOPP_DECODE_CASE(__nv_bfloat16, 64, true)
+        }
+        if (D == 128) { YOCOPP_DECODE_CASE(float, 128, true) }
+        YOCOPP_DECODE_CASE(float, 64, true)
     }
     if (cache->dtype == YOCOPP_BF16) {
-        if (D == 128) { YOCOPP_DECODE_CASE(__nv_bfloat16, 128) }
-        YOCOPP_DECODE_CASE(__nv_bfloat16, 64)
+        if (D == 128) { YOCOPP_DECODE_CASE(__nv_bfloat16, 128, false) }
+        YOCOPP_DECODE_CASE(__nv_bfloat16, 64, false)
     }
-    if (D == 128) { YOCOPP_DECODE_CASE(float, 128) }
-    YOCOPP_DECODE_CASE(float, 64)
+    if (D == 128) { YOCOPP_DECODE_CASE(float, 128, false) }
+    YOCOPP_DECODE_CASE(float, 64, false)
 #undef YOCOPP_DECODE_CASE
 }
 
@@ -418,6 +458,21 @@ int32_t yocopp_decode_attn_partial(const void* q, const yocopp_cache* cache, con
     if (partial == nullptr) return YOCOPP_EINVAL;
     return decode_attn_impl(q, cache, seq_lens, nullptr, partial, num_q_heads, scale, workspace,
                             workspace_bytes, stream);
+}
+
+int32_t yocopp_decode_attn_fused(const void* q, const yocopp_cache* cache_i, const yocopp_cache* cache_1,
+                                 const float alpha[4], float lambda, const int32_t* seq_lens, void* out,
+                                 int32_t num_q_heads, float scale, void* workspace, int64_t workspace_bytes,
+                                 void* stream) {
+    if (out == nullptr || alpha == nullptr || cache_1 == nullptr) return YOCOPP_EINVAL;
+    if (!std::isfinite(lambda) || !std::isfinite(alpha[0]) || !std::isfinite(alpha[1]) ||
+        !std::isfinite(alpha[2]) || !std::isfinite(alpha[3]))
+        return YOCOPP_EINVAL;
+    FusedArgs f;
+    f.cache1 = cache_1;
+    for (int j = 0; j < 4; ++j) f.coef[j] = lambda * alpha[j];
+    return decode_attn_impl(q, cache_i, seq_lens, out, nullptr, num_q_heads, scale, workspace, workspace_bytes,
+                            stream, &f);
 }
 
 int32_t yocopp_decode_combine(const float* partials, int32_t num_parts, int64_t rows, int32_t head_dim,

@@ -165,6 +165,25 @@ int32_t yocopp_decode_attn(const void* q, const yocopp_cache* cache, const int32
                            int64_t workspace_bytes, void* stream);
 
 /*
+ * yocopp_decode_attn_fused - the read-time alternative the composition is
+ * designed to avoid (YOCO++, section 1 on FusedKV and section 3: combining
+ * several layers' KVs while decoding costs extra I/O; composing before the
+ * cache write keeps decoding at one KV set per layer).  Same attention as
+ * yocopp_decode_attn over K' = lambda (alpha[0] K_1 + alpha[1] K_i) and
+ * V' = lambda (alpha[2] V_1 + alpha[3] V_i), but K', V' are formed in fp32
+ * at read time (never rounded to the cache type) from two RAW caches, so
+ * every decode step reads twice the bytes.  The exact FusedKV combination is
+ * not given by the pages; this is the YOCO++ formula evaluated at read time.
+ *   cache_i : raw K_i, V_i of layer L/2;  cache_1 : raw K_1, V_1 of layer 1;
+ *             identical shape, dtype, layout and block table.
+ * Other arguments as yocopp_decode_attn (its workspace size applies).
+ */
+int32_t yocopp_decode_attn_fused(const void* q, const yocopp_cache* cache_i, const yocopp_cache* cache_1,
+                                 const float alpha[4], float lambda, const int32_t* seq_lens, void* out,
+                                 int32_t num_q_heads, float scale, void* workspace, int64_t workspace_bytes,
+                                 void* stream);
+
+/*
  * yocopp_decode_attn_partial - yocopp_decode_attn over this caller's cached
  * positions only, kept unnormalised so that it can be merged with results
  * over other positions of the same sequences (for example other GPUs' shards
