@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--decode-kernel", type=int, default=0, choices=[0, 1, 2],
+                    help="score product of the decode kernel: 0 default (= 2), 1 CUDA cores, 2 tcgen05 tensor cores")
     ap.add_argument("--compose-layers", type=int, default=0,
                     help="profiling only: compose just the last N self-decoder layers (0 = all)")
     ap.add_argument("--cross-layers", type=int, default=0,
@@ -77,7 +79,16 @@ KERNEL_SOURCES = {
                               "decode_attention_yocopp_b200/csrc/common.cuh"],
     "decode_split_kernel": ["decode_attention_yocopp_b200/csrc/decode_attn.cuh",
                             "decode_attention_yocopp_b200/csrc/common.cuh"],
+    "decode_tc_kernel": ["decode_attention_yocopp_b200/csrc/decode_attn_tc.cuh",
+                         "decode_attention_yocopp_b200/csrc/decode_attn.cuh",
+                         "decode_attention_yocopp_b200/csrc/common.cuh"],
 }
+
+
+def decode_kernel_name(w, which: int) -> str:
+    """The decode kernel the library dispatches for this workload (mirrors the C-ABI rule)."""
+    tc = which != 1 and w.dtype == "bf16" and w.d == 128
+    return "decode_tc_kernel" if tc else "decode_split_kernel"
 
 
 def ncu_traffic(kernel: str, workload: str):
@@ -328,6 +339,7 @@ def run_ours(args, rank, world, local):
     import decode_attention_yocopp_b200 as y
     y.load()
     y.yocopp_get_device_status(reset=True)
+    y.yocopp_set_decode_kernel(args.decode_kernel)
     w = rank_workload(args.config, rank)
     comp_layers, cross_layers = trim(w, args)
     step = Step(w, comp_layers, cross_layers)
@@ -432,9 +444,10 @@ def run_ours(args, rank, world, local):
                  "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(ach_comp / peak, 4),
                  "traffic": ncu_traffic("compose_append_kernel", workload),
                  "algorithmic_bytes_per_launch": w.compose_bytes(w.total_prefill)}
-    roof_attn = {"kernel": "decode_split_kernel (one layer, split + merge)", "bound": "hbm",
+    dk = decode_kernel_name(w, args.decode_kernel)
+    roof_attn = {"kernel": f"{dk} (one layer, split + merge)", "bound": "hbm",
                  "achieved": round(ach_attn, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                 "frac": round(ach_attn / peak, 4), "traffic": ncu_traffic("decode_split_kernel", workload),
+                 "frac": round(ach_attn / peak, 4), "traffic": ncu_traffic(dk, workload),
                  "algorithmic_bytes_per_launch": kv_bytes_layer}
     dominant = roof_comp if t_prefill >= t_attn else roof_attn
     line = {
@@ -446,6 +459,7 @@ def run_ours(args, rank, world, local):
                    "head_dim": w.d, "paged": w.paged, "parallelism": f"dp{world} (sequences per rank, no exchange)",
                    "l2": "inputs larger than L2 (shared cache and per-step compose streams exceed 126 MB)"},
         "kv_read_frac_of_peak": round(value / world / peak, 4),
+        "decode_kernel": decode_kernel_name(w, args.decode_kernel),
         "compose_gbs": round(compose_gbs, 1),
         "compose_frac_of_peak": round(compose_gbs / world / peak, 4),
         "decode_tok_s": round(tok_all / (t_decode_max * 1e-3), 1),

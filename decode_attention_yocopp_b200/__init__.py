@@ -30,7 +30,7 @@ YOCOPP_F32 = 1
 EXPORTS = ("yocopp_compose_append", "yocopp_decode_attn_workspace_size", "yocopp_decode_attn",
            "yocopp_get_device_status", "yocopp_status_string", "yocopp_version",
            "yocopp_testing_set_decode_fault", "yocopp_decode_attn_static", "yocopp_decode_attn_partial",
-           "yocopp_decode_combine", "yocopp_decode_attn_fused")
+           "yocopp_decode_combine", "yocopp_decode_attn_fused", "yocopp_set_decode_kernel")
 
 
 class yocopp_cache(ctypes.Structure):
@@ -76,6 +76,8 @@ def load(path: Optional[str] = None):
     lib.yocopp_testing_set_decode_fault.argtypes = [I32, I64]
     lib.yocopp_decode_attn_partial.restype = I32
     lib.yocopp_decode_attn_partial.argtypes = [V, ctypes.POINTER(yocopp_cache), V, V, I32, ctypes.c_float, V, I64, V]
+    lib.yocopp_set_decode_kernel.restype = I32
+    lib.yocopp_set_decode_kernel.argtypes = [I32]
     lib.yocopp_decode_attn_fused.restype = I32
     lib.yocopp_decode_attn_fused.argtypes = [V, ctypes.POINTER(yocopp_cache), ctypes.POINTER(yocopp_cache),
                                              ctypes.POINTER(ctypes.c_float), ctypes.c_float, V, V, I32,
@@ -191,6 +193,14 @@ def yocopp_decode_attn_partial(q, cache: yocopp_cache, seq_lens, partial, worksp
                                            workspace.numel() * workspace.element_size() if workspace is not None else 0,
                                            _stream(stream))
     _check("yocopp_decode_attn_partial", rc)
+
+
+DECODE_DEFAULT, DECODE_CUDA_CORES, DECODE_TENSOR_CORES = 0, 1, 2
+
+
+def yocopp_set_decode_kernel(which: int) -> None:
+    """Choose the score product of later decode launches (0 default, 1 CUDA cores, 2 tcgen05)."""
+    _check("yocopp_set_decode_kernel", load().yocopp_set_decode_kernel(int(which)))
 
 
 def yocopp_decode_attn_fused(q, cache_i: yocopp_cache, cache_1: yocopp_cache, alpha: Sequence[float], lam: float,

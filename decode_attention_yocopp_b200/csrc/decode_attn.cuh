@@ -1,4 +1,6 @@
-// Split-K GQA decode attention over the shared cross-decoder cache.
+// Split-K GQA decode attention over the shared cross-decoder cache
+// (CUDA-core score product; decode_attn_tc.cuh moves the scores to tcgen05
+// for bf16 / head_dim 128 and reuses this file's merge and helpers).
 //
 // You Only Cache Once (abstract): the cross-decoder reuses the self-decoder's
 // cache through cross-attention.  YOCO++ section 2: every upper-half layer
@@ -426,9 +428,8 @@ struct ConsumerWarp {
 // then each thread accumulates 4 channels with 16-byte loads.
 template <typename T, int D, int G, int W, typename Sync>
 __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c0, int c1, int64_t out_row0,
-                                            float* scratch, int scratch_floats, Sync& sync) {
+                                            float* scratch, int scratch_floats, Sync& sync, int tid) {
     constexpr int NT = W * 32;
-    const int tid = threadIdx.x;
     const int nparts = c1 - c0 + 1;
     const int cap = (scratch_floats - 2 * G) / (2 * G);  // parts that fit the staging area
     const float* pm = p.ws_m + int64_t(bg + c0) * G;
@@ -498,6 +499,66 @@ __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c
         }
     }
     return ok;
+}
+
+// End of a (sequence, kv-head) segment, after the warps' states are stashed in
+// mg_*: merge them; write the output (whole plane) or this CTA's partial, then
+// arrive on the plane's counter and, as the last CTA, merge the plane.  Run by
+// the W consumer warps (ctid = consumer thread index).  False on a timed-out
+// rendezvous.
+template <typename T, int D, int G, int W, typename Sync>
+__device__ __forceinline__ bool flush_segment(const DecodeParams& p, const TileMeta& mt, int ctid, int tpc,
+                                              const int* s_ts, float* mg_m, float* mg_l, float* mg_o, float* scratch,
+                                              int scratch_floats, Sync& consumer_sync, int& s_last) {
+    if (!consumer_sync()) return false;
+    const int bg = mt.b * p.hkv + mt.g;
+    const int slot = bg + int(blockIdx.x);
+    const bool whole = mt.flags & kWhole;
+    for (int idx = ctid; idx < G * D; idx += W * 32) {
+        const int h = idx / D, c = idx % D;
+        float M = NEG_INF_F;
+#pragma unroll
+        for (int w2 = 0; w2 < W; ++w2) M = fmaxf(M, mg_m[w2 * G + h]);
+        float Ls = 0.f, O = 0.f;
+        if (M != NEG_INF_F) {
+#pragma unroll
+            for (int w2 = 0; w2 < W; ++w2) {
+                const float f = exp2f(mg_m[w2 * G + h] - M);
+                Ls += f * mg_l[w2 * G + h];
+                O += f * mg_o[(w2 * G + h) * D + c];
+            }
+        }
+        if (whole) {
+            emit<T, D>(p, int64_t(mt.b) * p.hq + mt.g * G + h, c, M, Ls, O);
+        } else {
+            p.ws_o[(int64_t(slot) * G + h) * D + c] = O;
+            if (c == 0) {
+                p.ws_m[int64_t(slot) * G + h] = M;
+                p.ws_l[int64_t(slot) * G + h] = Ls;
+            }
+        }
+    }
+    if (!whole) {
+        // publish this CTA's partial, count arrivals; the last CTA merges the plane
+        __threadfence();
+        if (!consumer_sync()) return false;
+        const int nt = ntiles_of(mt.len, mt.pad);  // pad carries the kernel's tile size
+        const int first = s_ts[mt.b] + mt.g * nt;
+        const int c0 = first / tpc, c1 = (first + nt - 1) / tpc;
+        if (ctid == 0) {
+            const unsigned arrived = arrive_plane(p.ws_cnt + bg, p.epoch);
+            if (arrived == 0) record_status(YOCOPP_EWORKSPACE);
+            s_last = arrived == unsigned(c1 - c0 + 1);
+            __threadfence();
+        }
+        if (!consumer_sync()) return false;
+        if (s_last) {
+            if (!merge_plane<T, D, G, W>(p, bg, c0, c1, int64_t(mt.b) * p.hq + mt.g * G, scratch, scratch_floats,
+                                         consumer_sync, ctid))
+                return false;
+        }
+    }
+    return consumer_sync();
 }
 
 template <typename T, int D, int G, int W, int STAGES, int CTAS_PER_SM, bool FUSED>
@@ -616,7 +677,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                 m.k = __shfl_sync(0xffffffffu, k, j);
                 m.len = __shfl_sync(0xffffffffu, len, j);
                 m.flags = __shfl_sync(0xffffffffu, flags, j);
-                m.pad = 0;
+                m.pad = TILE;  // the tile size, for the plane's tile count at flush
                 int r[NSB_MAX];
 #pragma unroll
                 for (int s = 0; s < NSB_MAX; ++s) r[s] = __shfl_sync(0xffffffffu, rows[s], j);
@@ -727,70 +788,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         if (mt.flags & kLast) {
             // ---- end of segment: merge the warps' states, emit output or a partial
             cw.stash(mg_m, mg_l, mg_o);
-            if (!consumer_sync()) {
-                record_status(YOCOPP_ETIMEOUT);
-                s_abort = 1;
-                break;
-            }
-            const int bg = mt.b * p.hkv + mt.g;
-            const int slot = bg + int(blockIdx.x);
-            const bool whole = mt.flags & kWhole;
-            for (int idx = tid; idx < G * D; idx += W * 32) {
-                const int h = idx / D, c = idx % D;
-                float M = NEG_INF_F;
-#pragma unroll
-                for (int w2 = 0; w2 < W; ++w2) M = fmaxf(M, mg_m[w2 * G + h]);
-                float Ls = 0.f, O = 0.f;
-                if (M != NEG_INF_F) {
-#pragma unroll
-                    for (int w2 = 0; w2 < W; ++w2) {
-                        const float f = exp2f(mg_m[w2 * G + h] - M);
-                        Ls += f * mg_l[w2 * G + h];
-                        O += f * mg_o[(w2 * G + h) * D + c];
-                    }
-                }
-                if (whole) {
-                    emit<T, D>(p, int64_t(mt.b) * p.hq + mt.g * G + h, c, M, Ls, O);
-                } else {
-                    p.ws_o[(int64_t(slot) * G + h) * D + c] = O;
-                    if (c == 0) {
-                        p.ws_m[int64_t(slot) * G + h] = M;
-                        p.ws_l[int64_t(slot) * G + h] = Ls;
-                    }
-                }
-            }
-            if (!whole) {
-                // publish this CTA's partial, count arrivals; the last CTA merges the plane
-                __threadfence();
-                if (!consumer_sync()) {
-                    record_status(YOCOPP_ETIMEOUT);
-                    s_abort = 1;
-                    break;
-                }
-                const int nt = ntiles_of(mt.len, TILE);
-                const int first = s_ts[mt.b] + mt.g * nt;
-                const int c0 = first / tpc, c1 = (first + nt - 1) / tpc;
-                if (tid == 0) {
-                    const unsigned arrived = arrive_plane(p.ws_cnt + bg, p.epoch);
-                    if (arrived == 0) record_status(YOCOPP_EWORKSPACE);
-                    s_last = arrived == unsigned(c1 - c0 + 1);
-                    __threadfence();
-                }
-                if (!consumer_sync()) {
-                    record_status(YOCOPP_ETIMEOUT);
-                    s_abort = 1;
-                    break;
-                }
-                if (s_last) {
-                    if (!merge_plane<T, D, G, W>(p, bg, c0, c1, int64_t(mt.b) * p.hq + mt.g * G, p_s,
-                                                 int((L::kTileStart - L::kP) / sizeof(float)), consumer_sync)) {
-                        record_status(YOCOPP_ETIMEOUT);
-                        s_abort = 1;
-                        break;
-                    }
-                }
-            }
-            if (!consumer_sync()) {
+            if (!flush_segment<T, D, G, W>(p, mt, tid, tpc, s_ts, mg_m, mg_l, mg_o, p_s,
+                                           int((L::kTileStart - L::kP) / sizeof(float)), consumer_sync, s_last)) {
                 record_status(YOCOPP_ETIMEOUT);
                 s_abort = 1;
                 break;

@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "compose_append.cuh"
 #include "decode_attn.cuh"
+#include "decode_attn_tc.cuh"
 
 namespace yocopp {
 namespace {
@@ -20,6 +21,7 @@ constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
 
 int g_test_drop_tile = -1;
+int g_decode_kernel = 0;  // 0 / 2: tensor-core scores where supported, 1: CUDA-core scores
 
 // Per-call tag for the decode kernel's arrival counters: strictly increasing
 // within the process, 44 bits, never 0 (a zero-filled counter is older than
@@ -68,9 +70,9 @@ EncodeFn encode_fn() {
     return fn;
 }
 
-// 2-D view of a cache tensor: rows of head_dim elements; 128-byte swizzled
-// boxes of (128 / elem) x box_rows.
-bool encode_rows(CUtensorMap* map, void* base, int dtype, int head_dim, int64_t rows, int box_rows) {
+// 2-D view of a cache (or query) tensor: rows of head_dim elements; 128-byte
+// swizzled boxes of (128 / elem) x box_rows.
+bool encode_rows(CUtensorMap* map, const void* base, int dtype, int head_dim, int64_t rows, int box_rows) {
     EncodeFn fn = encode_fn();
     if (!fn) return false;
     const int eb = elem_bytes(dtype);
@@ -79,7 +81,7 @@ bool encode_rows(CUtensorMap* map, void* base, int dtype, int head_dim, int64_t 
     cuuint32_t box[2] = {cuuint32_t(128 / eb), cuuint32_t(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     return fn(map, dtype == YOCOPP_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
-              base, gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -182,6 +184,41 @@ int32_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const CUtens
     return cuda_status(cudaLaunchKernelEx(&lc, kern, tk, tv, tk1, tv1, p));
 }
 
+template <int G>
+int32_t launch_decode_tc(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq, const DecodeParams& p,
+                         cudaStream_t st) {
+    constexpr int STAGES = 3;
+    auto kern = decode_tc_kernel<G, STAGES>;
+    const size_t smem = TcSmem<G, STAGES>::bytes(p.batch);
+    static bool attr_set[kMaxDevices] = {false};
+    static size_t max_dyn[kMaxDevices] = {0};
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return YOCOPP_ECUDA;
+    if (!attr_set[dev]) {
+        int maxopt = 0;
+        cudaFuncAttributes fa;
+        if (cudaDeviceGetAttribute(&maxopt, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+            cudaFuncGetAttributes(&fa, kern) != cudaSuccess)
+            return YOCOPP_ECUDA;
+        max_dyn[dev] = size_t(maxopt) - fa.sharedSizeBytes;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(max_dyn[dev])) != cudaSuccess)
+            return YOCOPP_ECUDA;
+        attr_set[dev] = true;
+    }
+    if (smem > max_dyn[dev]) return YOCOPP_EINVAL;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(unsigned(p.num_ctas), 1, 1);
+    lc.blockDim = dim3(192, 1, 1);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&lc, kern, tk, tv, tq, p));
+}
+
 struct WorkspaceLayout {
     size_t cnt, m, l, o, total;
 };
@@ -269,6 +306,12 @@ int32_t yocopp_get_device_status(int32_t reset) {
         if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return YOCOPP_ECUDA;
     }
     return v;
+}
+
+int32_t yocopp_set_decode_kernel(int32_t which) {
+    if (which < 0 || which > 2) return YOCOPP_EINVAL;
+    g_decode_kernel = which;
+    return YOCOPP_OK;
 }
 
 int32_t yocopp_testing_set_decode_fault(int32_t drop_tile, int64_t wait_limit_ns) {
@@ -366,13 +409,17 @@ static int32_t decode_attn_impl(const void* q, const yocopp_cache* cache, const 
     if (!(scale >= 0.f) || !std::isfinite(scale)) return YOCOPP_EINVAL;
     const int sms = sm_count(current_device());
     if (sms <= 0) return YOCOPP_ECUDA;
-    const int num_ctas = sms * YOCOPP_DECODE_CTAS_PER_SM;
+    // tensor-core scores: bf16, head_dim 128, no read-time composition, block size >= 16, and the
+    // batch's tile table fits next to the 3-stage ring
+    const bool use_tc = g_decode_kernel != 1 && fused == nullptr && cache->dtype == YOCOPP_BF16 &&
+                        cache->head_dim == 128 && TcSmem<4, 3>::bytes(cache->batch) <= 232448 - 1024;
+    const int num_ctas = use_tc ? sms : sms * YOCOPP_DECODE_CTAS_PER_SM;
     const WorkspaceLayout wl = workspace_layout(cache->batch, cache->num_kv_heads, G, cache->head_dim, num_ctas);
     if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < int64_t(wl.total))
         return YOCOPP_EWORKSPACE;
 
     const int D = cache->head_dim;
-    const int tile = ((D * elem_bytes(cache->dtype)) <= 256 ? 64 : 32) / (fused != nullptr ? 2 : 1);
+    const int tile = use_tc ? TcShape::TILE : ((D * elem_bytes(cache->dtype)) <= 256 ? 64 : 32) / (fused != nullptr ? 2 : 1);
     const bool paged = cache->block_table != nullptr;
     const int boxr = paged ? (cache->block_size < tile ? cache->block_size : tile) : tile;
     const int64_t rows = paged ? int64_t(cache->num_blocks) * cache->num_kv_heads * cache->block_size
@@ -420,6 +467,17 @@ static int32_t decode_attn_impl(const void* q, const yocopp_cache* cache, const 
     p.fa1v = fused ? fused->coef[2] : 0.f;
     p.fa2v = fused ? fused->coef[3] : 0.f;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    if (use_tc) {
+        alignas(64) CUtensorMap tq;
+        if (!encode_rows(&tq, q, cache->dtype, D, int64_t(cache->batch) * num_q_heads, TcShape::QROWS))
+            return YOCOPP_ECUDA;
+        switch (G) {
+            case 1: return launch_decode_tc<1>(tk, tv, tq, p, st);
+            case 2: return launch_decode_tc<2>(tk, tv, tq, p, st);
+            default: return launch_decode_tc<4>(tk, tv, tq, p, st);
+        }
+    }
 
 #define YOCOPP_DECODE_CASE(TT, DD, FF)                                                 \
     switch (G) {                                                                       \

@@ -254,6 +254,19 @@ const char* yocopp_status_string(int32_t status);
 int32_t yocopp_version(void);
 
 /*
+ * yocopp_set_decode_kernel - which score product later yocopp_decode_attn /
+ * _partial / _static launches use (process-wide, host-side):
+ *   0  the default, which is 2;
+ *   1  CUDA-core packed fp32 FMA for q.k (every dtype and head_dim);
+ *   2  tcgen05 tensor cores for the query-group x key-tile product where
+ *      supported (bf16, head_dim 128, batch up to about 2400; otherwise the
+ *      CUDA-core kernel runs).
+ * Both give the same results within rounding; the value sum and the softmax
+ * run on the CUDA cores in both.  Returns YOCOPP_EINVAL for other values.
+ */
+int32_t yocopp_set_decode_kernel(int32_t which);
+
+/*
  * yocopp_testing_set_decode_fault - failure-injection hook for tests.
  * Host-side, process-wide; affects later yocopp_decode_attn launches.
  *   drop_tile     : index (in the split plan's flattened tile order) of one

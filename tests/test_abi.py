@@ -76,3 +76,11 @@ def test_more_host_checks():
     assert lib.yocopp_decode_attn(0x10, ctypes.byref(c), 0x10, 0x10, 24, 0.0, 0x100, 1 << 20, None) == y.YOCOPP_EINVAL
     assert lib.yocopp_decode_attn(0x10, ctypes.byref(c), 0x10, 0x10, 12, 0.0, 0x100, 1 << 20, None) == y.YOCOPP_EINVAL
     assert lib.yocopp_testing_set_decode_fault(-1, 0) == y.YOCOPP_EINVAL
+
+
+def test_decode_kernel_selector():
+    lib = y.load()
+    for which in (0, 1, 2, 0):
+        assert lib.yocopp_set_decode_kernel(which) == y.YOCOPP_OK
+    assert lib.yocopp_set_decode_kernel(3) == y.YOCOPP_EINVAL
+    assert lib.yocopp_set_decode_kernel(-1) == y.YOCOPP_EINVAL

@@ -1,4 +1,6 @@
-"""GPU parity of yocopp_decode_attn against the fp64 oracle, on the same cache bytes.
+"""GPU parity of yocopp_decode_attn against the fp64 oracle, on the same cache bytes
+(default kernel: tcgen05 scores for bf16 / head_dim 128, the CUDA-core kernel
+otherwise; test_gpu_decode_cuda_cores.py reruns these with CUDA-core scores).
 
 You Only Cache Once (abstract): the cross-decoder reuses the cached keys and
 values through cross-attention; YOCO++ section 2: all upper-half layers read
@@ -96,7 +98,11 @@ def run_case(y, orc, *, dtype, d, hkv, G, lens, paged=False, block_size=64, key_
     return got, ref
 
 
-EDGE_LENS = [0, 1, 63, 64, 65, 4097]
+EDGE_LENS = [0, 1, 63, 64, 65, 127, 128, 129, 4097]
+
+
+def test_single_small_tile(y, orc):
+    run_case(y, orc, dtype="bf16", d=128, hkv=1, G=4, lens=[100])
 
 
 def test_edge_lengths_contiguous(y, orc):
