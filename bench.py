@@ -403,6 +403,20 @@ def run_ours(args, rank, world, local):
     t_self = sum(a.elapsed_time(b) for a, b in zip(evf["b"], evf["c"]))
     t_full_max = max_over_ranks(t_full, world)
     t_self_max = max_over_ranks(t_self, world)
+    # the same decode step captured once in a CUDA graph and replayed
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step.run_decode_full()
+    graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    ga = _event()
+    for _ in range(K):
+        graph.replay()
+    gb = _event()
+    torch.cuda.synchronize()
+    t_graph_max = max_over_ranks(ga.elapsed_time(gb), world)
+    del graph
     self_bytes = sum_over_ranks(w.kv_bytes() * len(step.selfl) * K, world)
 
     # contrast: the same cross-decoder layers composing K', V' at read time (2x the bytes)
@@ -467,6 +481,8 @@ def run_ours(args, rank, world, local):
         "decode_full_step": {"tok_s": round(tok_all / (t_full_max * 1e-3), 1),
                              "ms_per_step": round(t_full_max / K, 4),
                              "self_attn_kv_gbs": round(self_bytes / (t_self_max * 1e-3) / 1e9, 1),
+                             "cuda_graph_tok_s": round(tok_all / (t_graph_max * 1e-3), 1),
+                             "cuda_graph_ms_per_step": round(t_graph_max / K, 4),
                              "what": "decoded token appended to layers 1..L/2, L/2 self-decoder attentions over "
                                      "their own caches, L/2 cross-decoder attentions over the shared cache"},
         "read_time_composition_contrast": {

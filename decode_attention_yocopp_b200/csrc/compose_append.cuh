@@ -8,9 +8,8 @@
 //
 // The kernel is a pure HBM stream: per (token, head) row it reads four input
 // rows and writes two cache rows.  Each thread moves 16-byte chunks with
-// 128-bit loads (read-once, no L1 allocation) and stores 128 bits; a grid-
-// stride loop over a grid sized to the SM count keeps two chunks per thread
-// in flight.
+// 128-bit loads (read-once, no L1 allocation) and stores 128 bits, in a
+// grid-stride loop over a grid of one 1024-thread CTA per SM.
 //
 // Arithmetic.  The weighted sum a1*x1 + a2*xi can cancel almost completely
 // (x1, xi ~ N(0,1) and |a1| ~ |a2|), and a plain fp32 evaluation then loses
@@ -119,10 +118,24 @@ __device__ __forceinline__ int64_t cache_row_offset(const ComposeParams& p, int 
     return ((int64_t(blk) * p.hkv + h) * p.block_size + position % p.block_size) * ROWB;
 }
 
+// Launch shape (compile-time; the defaults are the measured best on B200).
+// One 1024-thread CTA per SM, one chunk per thread per iteration: the grid is
+// exactly resident (no second-wave tail), and each iteration of the grid-
+// stride loop sweeps 148 x 1024 consecutive chunks of every stream.
+#ifndef YOCOPP_COMPOSE_THREADS
+#define YOCOPP_COMPOSE_THREADS 1024
+#endif
+#ifndef YOCOPP_COMPOSE_UNROLL
+#define YOCOPP_COMPOSE_UNROLL 1
+#endif
+#ifndef YOCOPP_COMPOSE_CTAS_PER_SM
+#define YOCOPP_COMPOSE_CTAS_PER_SM 1
+#endif
+
 template <typename T, int ROWB>
-__global__ void __launch_bounds__(256) compose_append_kernel(ComposeParams p) {
-    constexpr int CPR = ROWB / 16;  // 16-byte chunks per (token, head) row
-    constexpr int U = 2;            // chunks in flight per thread
+__global__ void __launch_bounds__(YOCOPP_COMPOSE_THREADS) compose_append_kernel(ComposeParams p) {
+    constexpr int CPR = ROWB / 16;                 // 16-byte chunks per (token, head) row
+    constexpr int U = YOCOPP_COMPOSE_UNROLL;       // chunks in flight per thread
     extern __shared__ int s_cu[];   // staged prefix offsets (ragged batches only)
 
     if (p.cu_new != nullptr) {

@@ -41,6 +41,7 @@ struct DecodeParams {
     uint8_t* out;
     const int32_t* seq_lens;
     const int32_t* block_table;  // nullptr: contiguous cache
+    unsigned long long* ws_gen;  // workspace header: [0] generation of the last finished call, [1] call arrivals
     unsigned long long* ws_cnt;  // [batch * hkv] arrival counters: (call epoch << 20) | CTAs arrived
     float* ws_m;                 // [slots][G]
     float* ws_l;                 // [slots][G]
@@ -50,7 +51,6 @@ struct DecodeParams {
     int32_t num_ctas;
     int32_t drop_tile;           // testing: a tile whose load is never issued (-1: none)
     uint64_t wait_limit_ns;
-    unsigned long long epoch;    // grows with every call (44 bits, never 0): tags this call's arrivals
     float* part_out;             // non-null: write unnormalised [batch][hq][D + 2] (o, m, l) instead of out
     float fa1k, fa2k, fa1v, fa2v;  // read-time composition (fused variant): lambda * alpha
 };
@@ -171,12 +171,32 @@ struct DecodeSmem {
     static size_t bytes(int batch) { return 1024 + kTileStart + size_t(batch + 1) * sizeof(int); }
 };
 
+// This call's epoch, read from the workspace header by each CTA at start.
+// header[0] = the epoch of the last call that every CTA joined (0 in a
+// zero-filled workspace); header[1] = (epoch << 20) | CTAs of the current call
+// that have read it.  Each CTA reads header[0], takes epoch = header[0] + 1,
+// and arrives on header[1]; the last CTA to arrive publishes the epoch in
+// header[0] for the next call.  Every CTA arrives right after reading, before
+// any work that could time out, so each call advances the epoch exactly once;
+// the epoch lives on the device, so a captured CUDA graph replays correctly.
+__device__ __forceinline__ unsigned long long join_call(unsigned long long* hdr, unsigned num_ctas) {
+    const unsigned long long epoch = __ldcg(hdr) + 1ull;
+    __threadfence();
+    atomicMax(hdr + 1, epoch << 20);
+    const unsigned long long old = atomicAdd(hdr + 1, 1ull);
+    if ((old >> 20) == epoch && unsigned(old & 0xFFFFFull) + 1u == num_ctas) {
+        __threadfence();
+        atomicMax(hdr, epoch);
+    }
+    return epoch;
+}
+
 // Arrive on a plane's counter for this call; returns how many CTAs have arrived
 // (this one included), or 0 if the counter holds a later call's tag (a
 // workspace that was not zero-filled before its first use).  The word is
-// (epoch << 20) | count.  Epochs only grow within a process, so atomicMax
-// replaces a tag left by any earlier call (finished or aborted) with this
-// call's tag and a zero count; two single atomics, no retry loop.
+// (epoch << 20) | count.  Epochs only grow, so atomicMax replaces a tag left by
+// any earlier call (finished or aborted) with this call's tag and a zero
+// count; two single atomics, no retry loop.
 __device__ __forceinline__ unsigned arrive_plane(unsigned long long* cnt, unsigned long long epoch) {
     atomicMax(cnt, epoch << 20);
     const unsigned long long old = atomicAdd(cnt, 1ull);
@@ -509,7 +529,8 @@ __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c
 template <typename T, int D, int G, int W, typename Sync>
 __device__ __forceinline__ bool flush_segment(const DecodeParams& p, const TileMeta& mt, int ctid, int tpc,
                                               const int* s_ts, float* mg_m, float* mg_l, float* mg_o, float* scratch,
-                                              int scratch_floats, Sync& consumer_sync, int& s_last) {
+                                              int scratch_floats, Sync& consumer_sync, int& s_last,
+                                              unsigned long long epoch) {
     if (!consumer_sync()) return false;
     const int bg = mt.b * p.hkv + mt.g;
     const int slot = bg + int(blockIdx.x);
@@ -546,7 +567,7 @@ __device__ __forceinline__ bool flush_segment(const DecodeParams& p, const TileM
         const int first = s_ts[mt.b] + mt.g * nt;
         const int c0 = first / tpc, c1 = (first + nt - 1) / tpc;
         if (ctid == 0) {
-            const unsigned arrived = arrive_plane(p.ws_cnt + bg, p.epoch);
+            const unsigned arrived = arrive_plane(p.ws_cnt + bg, epoch);
             if (arrived == 0) record_status(YOCOPP_EWORKSPACE);
             s_last = arrived == unsigned(c1 - c0 + 1);
             __threadfence();
@@ -602,7 +623,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     // from the previous kernel until this wait returns
     griddep_wait();
     griddep_launch_dependents();
+    __shared__ unsigned long long s_epoch;
+    if (tid == 0) s_epoch = join_call(p.ws_gen, gridDim.x);
     tile_prefix<TILE>(p, s_ts, s_warp);  // ends with __syncthreads()
+    const unsigned long long epoch = s_epoch;
     // sequences with no cached positions: zero output (CTA b mod grid writes it)
     for (int b = blockIdx.x; b < p.batch; b += p.num_ctas) {
         if (s_ts[b + 1] != s_ts[b]) continue;
@@ -789,7 +813,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             // ---- end of segment: merge the warps' states, emit output or a partial
             cw.stash(mg_m, mg_l, mg_o);
             if (!flush_segment<T, D, G, W>(p, mt, tid, tpc, s_ts, mg_m, mg_l, mg_o, p_s,
-                                           int((L::kTileStart - L::kP) / sizeof(float)), consumer_sync, s_last)) {
+                                           int((L::kTileStart - L::kP) / sizeof(float)), consumer_sync, s_last,
+                                           epoch)) {
                 record_status(YOCOPP_ETIMEOUT);
                 s_abort = 1;
                 break;

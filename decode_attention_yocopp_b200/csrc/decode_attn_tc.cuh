@@ -232,7 +232,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     }
     griddep_wait();
     griddep_launch_dependents();
+    __shared__ unsigned long long s_epoch;
+    if (tid == 0) s_epoch = join_call(p.ws_gen, gridDim.x);
     tile_prefix<TILE>(p, s_ts, s_warp);  // ends with __syncthreads()
+    const unsigned long long epoch = s_epoch;
     for (int b = blockIdx.x; b < p.batch; b += p.num_ctas) {
         if (s_ts[b + 1] != s_ts[b]) continue;
         for (int idx = tid; idx < p.hq * S::D; idx += blockDim.x)
@@ -466,7 +469,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             cw.stash(mg_m, mg_l, mg_o);
             if (!flush_segment<__nv_bfloat16, S::D, G, W>(p, mt, ctid, tpc, s_ts, mg_m, mg_l, mg_o, p_s,
                                                           int((L::kTileStart - L::kP) / sizeof(float)),
-                                                          consumer_sync, s_last)) {
+                                                          consumer_sync, s_last, epoch)) {
                 record_status(YOCOPP_ETIMEOUT);
                 s_abort = 1;
                 break;

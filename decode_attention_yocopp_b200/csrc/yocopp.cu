@@ -5,7 +5,6 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
-#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -22,14 +21,6 @@ constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
 
 int g_test_drop_tile = -1;
 int g_decode_kernel = 0;  // 0 / 2: tensor-core scores where supported, 1: CUDA-core scores
-
-// Per-call tag for the decode kernel's arrival counters: strictly increasing
-// within the process, 44 bits, never 0 (a zero-filled counter is older than
-// every call).
-unsigned long long next_epoch() {
-    static std::atomic<unsigned long long> counter{0};
-    return (counter.fetch_add(1) + 1) & 0xFFFFFFFFFFFull;
-}
 uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -115,11 +106,12 @@ int32_t launch_compose(ComposeParams& p, cudaStream_t st) {
     const int sms = sm_count(dev);
     if (sms <= 0) return YOCOPP_ECUDA;
     const int64_t nchunks = p.total_rows * (ROWB / 16);
-    int64_t grid = (nchunks + 511) / 512;
-    if (grid > int64_t(sms) * 8) grid = int64_t(sms) * 8;
+    constexpr int64_t per_cta = int64_t(YOCOPP_COMPOSE_THREADS) * YOCOPP_COMPOSE_UNROLL;
+    int64_t grid = (nchunks + per_cta - 1) / per_cta;
+    if (grid > int64_t(sms) * YOCOPP_COMPOSE_CTAS_PER_SM) grid = int64_t(sms) * YOCOPP_COMPOSE_CTAS_PER_SM;
     if (grid < 1) grid = 1;
     const size_t smem = p.cu_new ? size_t(p.batch + 1) * sizeof(int) : 0;
-    compose_append_kernel<T, ROWB><<<unsigned(grid), 256, smem, st>>>(p);
+    compose_append_kernel<T, ROWB><<<unsigned(grid), YOCOPP_COMPOSE_THREADS, smem, st>>>(p);
     return cuda_status(cudaGetLastError());
 }
 
@@ -220,7 +212,7 @@ int32_t launch_decode_tc(const CUtensorMap& tk, const CUtensorMap& tv, const CUt
 }
 
 struct WorkspaceLayout {
-    size_t cnt, m, l, o, total;
+    size_t gen, cnt, m, l, o, total;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -228,8 +220,9 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 WorkspaceLayout workspace_layout(int batch, int hkv, int G, int D, int num_ctas) {
     const size_t slots = size_t(num_ctas) + size_t(batch) * hkv;
     WorkspaceLayout w;
-    w.cnt = 0;
-    w.m = up256(size_t(batch) * hkv * sizeof(unsigned long long));
+    w.gen = 0;                      // header: generation word + call-arrival word
+    w.cnt = 256;
+    w.m = w.cnt + up256(size_t(batch) * hkv * sizeof(unsigned long long));
     w.l = w.m + up256(slots * G * sizeof(float));
     w.o = w.l + up256(slots * G * sizeof(float));
     w.total = w.o + up256(slots * G * D * sizeof(float));
@@ -443,6 +436,7 @@ static int32_t decode_attn_impl(const void* q, const yocopp_cache* cache, const 
     p.out = static_cast<uint8_t*>(out);
     p.seq_lens = seq_lens;
     p.block_table = cache->block_table;
+    p.ws_gen = reinterpret_cast<unsigned long long*>(ws + wl.gen);
     p.ws_cnt = reinterpret_cast<unsigned long long*>(ws + wl.cnt);
     p.ws_m = reinterpret_cast<float*>(ws + wl.m);
     p.ws_l = reinterpret_cast<float*>(ws + wl.l);
@@ -460,7 +454,6 @@ static int32_t decode_attn_impl(const void* q, const yocopp_cache* cache, const 
     p.num_ctas = num_ctas;
     p.drop_tile = g_test_drop_tile;
     p.wait_limit_ns = g_wait_limit_ns;
-    p.epoch = next_epoch();
     p.part_out = part_out;
     p.fa1k = fused ? fused->coef[0] : 0.f;
     p.fa2k = fused ? fused->coef[1] : 0.f;

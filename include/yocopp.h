@@ -124,12 +124,13 @@ int32_t yocopp_compose_append(const void* K1, const void* V1, const void* Ki, co
  * yocopp_decode_attn needs for this cache shape and query-head count on the
  * current device (it depends on the device's SM count).  Returns a negative
  * yocopp_status on invalid arguments.  The workspace holds the per-split
- * partial softmax state (max, sum of exponentials, weighted value sum) and a
- * per-(sequence, kv-head) arrival counter tagged with a per-call value that
- * grows with every call.  Zero-fill the workspace once before its first use;
- * after that it never needs clearing, also not after a failed call.  (A
- * workspace that was never zero-filled can make a call report
- * YOCOPP_EWORKSPACE through yocopp_get_device_status.)
+ * partial softmax state (max, sum of exponentials, weighted value sum),
+ * per-(sequence, kv-head) arrival counters, and a call generation that the
+ * kernel itself advances (so calls captured in a CUDA graph replay
+ * correctly).  Zero-fill the workspace once before its first use; after that
+ * it never needs clearing, also not after a failed call.  (A workspace that
+ * was never zero-filled can make a call report YOCOPP_EWORKSPACE through
+ * yocopp_get_device_status.)
  */
 int64_t yocopp_decode_attn_workspace_size(const yocopp_cache* cache, int32_t num_q_heads);
 
