@@ -56,6 +56,35 @@ __device__ __forceinline__ float2 compose2(float2 x1, float2 xi, float2 na1, flo
     return ffma2(lam, s, fmul2(lam, lo));
 }
 
+// Rounding to bf16.  The fp32 value y from compose2 is within about one fp32
+// ulp of the exact composition, so converting it (nearest, ties to even)
+// rounds as the exact value does unless y lies within a few fp32 ulps of a
+// bf16 rounding midpoint: rounding to fp32 can carry a value onto a midpoint,
+// or (with the few-ulp slack) just past it.  Those values, about 5 in 2^16,
+// take the slow path: the composition in fp64, evaluated as written (inner
+// weighted sum, then lambda), rounded once to bf16.  The fp64 -> bf16 rounding
+// goes through fp32 with round-to-odd, which keeps a single rounding because
+// fp32 carries more than two extra bits (Boldo and Melquiond, "When double
+// rounding is odd", 2005).
+__device__ __forceinline__ bool near_bf16_midpoint(float y) {
+    return ((__float_as_uint(y) - 0x7FFEu) & 0xFFFFu) <= 4u;
+}
+
+__device__ __forceinline__ float f64_to_f32_round_odd(double v) {
+    float r;
+    asm("cvt.rz.f32.f64 %0, %1;" : "=f"(r) : "d"(v));
+    if (double(r) != v) r = __uint_as_float(__float_as_uint(r) | 1u);
+    return r;
+}
+
+__device__ __noinline__ uint32_t compose2_bf16_exact(float2 x1, float2 xi, float a1, float a2, float lam) {
+    const double ex = __dmul_rn(double(lam), __dadd_rn(__dmul_rn(double(a1), double(x1.x)),
+                                                        __dmul_rn(double(a2), double(xi.x))));
+    const double ey = __dmul_rn(double(lam), __dadd_rn(__dmul_rn(double(a1), double(x1.y)),
+                                                        __dmul_rn(double(a2), double(xi.y))));
+    return float2_to_bf16x2(f64_to_f32_round_odd(ex), f64_to_f32_round_odd(ey));
+}
+
 struct ComposeCoef {
     float2 a1, a2, na1, na2, lam;
 };
@@ -82,8 +111,12 @@ __device__ __forceinline__ uint4 compose_chunk<__nv_bfloat16>(uint4 a1, uint4 ai
     uint32_t* wr = reinterpret_cast<uint32_t*>(&r);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const float2 y = compose2(bf16x2_to_float2(w1[k]), bf16x2_to_float2(wi[k]), c.na1, c.na2, c.a1, c.a2, c.lam);
-        wr[k] = float2_to_bf16x2(y.x, y.y);
+        const float2 x1 = bf16x2_to_float2(w1[k]), xi = bf16x2_to_float2(wi[k]);
+        const float2 y = compose2(x1, xi, c.na1, c.na2, c.a1, c.a2, c.lam);
+        uint32_t w = float2_to_bf16x2(y.x, y.y);
+        if (near_bf16_midpoint(y.x) | near_bf16_midpoint(y.y))
+            w = compose2_bf16_exact(x1, xi, c.a1.x, c.a2.x, c.lam.x);
+        wr[k] = w;
     }
     return r;
 }

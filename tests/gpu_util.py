@@ -4,7 +4,8 @@ layouts built from logical [len][d] rows, and the parity tolerances.
 Tolerances (the bar each parity test asserts):
 * compose, bf16 cache: every stored value within 1 bf16 ulp of the oracle's
   fp64 composition rounded once to bf16 (ulp floored at the bf16 minimum
-  normal, 2^-126);
+  normal, 2^-126), and in fact bit-equal to that single rounding (the kernel
+  rounds the exact value, not an fp32 intermediate);
 * compose, fp32 cache: |gpu - exact| <= 4 * 2^-24 * (|lam a1 x1| + |lam a2 xi|),
   i.e. a few fp32 roundings of the two terms (the sum may cancel);
 * attention, bf16 output: against the oracle rounded to bf16, max |diff| <= 1e-2
@@ -59,12 +60,17 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
 
 
 def assert_compose_bf16(gpu_bits: np.ndarray, exact: np.ndarray, orc) -> None:
-    want = oracle.storage_to_f64(orc.round_to(exact, "bf16"), "bf16")
+    want_bits = orc.round_to(exact, "bf16")
+    want = oracle.storage_to_f64(want_bits, "bf16")
     got = oracle.storage_to_f64(gpu_bits, "bf16")
     diff = np.abs(got - want)
     lim = bf16_ulp(want)
     bad = np.nonzero(diff > lim)[0]
     assert bad.size == 0, f"{bad.size} composed values beyond 1 bf16 ulp; first {bad[:5]} got {got[bad[:5]]} want {want[bad[:5]]}"
+    # the kernel rounds the exact value once (ties to even), as the oracle does:
+    # the stored bits are the oracle's bits
+    neq = np.nonzero(np.asarray(gpu_bits, np.uint16) != np.asarray(want_bits, np.uint16))[0]
+    assert neq.size == 0, f"{neq.size} composed values not the single rounding; first {neq[:5]} got {got[neq[:5]]} want {want[neq[:5]]}"
 
 
 def assert_compose_f32(gpu: np.ndarray, x1: np.ndarray, xi: np.ndarray, a1: float, a2: float, lam: float, orc) -> None:

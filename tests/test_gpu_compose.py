@@ -181,3 +181,28 @@ def test_invalid_block_is_flagged(y, orc):
     kh = np_storage(kc)
     assert np.all(kh[1] == 0)
     assert np.all(kh[[0, 2, 3]] == BF16_NAN)
+
+
+@pytest.mark.parametrize("alpha", [(0.0, 1.5 / 35), (0.5 / 35, 1 / 35), (-0.75 / 35, 1.25 / 35)])
+def test_values_on_bf16_midpoints(y, orc, alpha):
+    """Weights whose compositions land on, or within a rounding error of, a bf16
+    rounding midpoint (35 * fp32(1.5/35) x is 1.5 x up to one part in 10^8, and
+    1.5 x of a bf16 value with an odd last bit has exactly one bit too many):
+    the stored value must be the single rounding of the exact composition."""
+    a1, a2 = (float(np.float32(v)) for v in alpha)
+    mags = np.arange(0x3F80, 0x4080, dtype=np.uint32)               # every bf16 value in [1, 4)
+    bits = np.concatenate([mags, mags | 0x8000]).astype(np.uint16)  # and its negative
+    rng = np.random.default_rng(11)
+    n = 64 * 128
+    xi = np.resize(bits, n).reshape(64, 1, 128)
+    x1 = rng.permutation(np.resize(bits, n)).reshape(64, 1, 128)
+    kc = torch.empty((1, 1, 64, 128), dtype=torch.bfloat16, device="cuda")
+    vc = torch.empty_like(kc)
+    cache = y.make_cache(kc, vc)
+    d1, di = to_device(x1, "bf16"), to_device(xi, "bf16")
+    y.yocopp_compose_append(d1, di, di, d1, (a1, a2, a1, a2), LAM, cache, torch.zeros(1, dtype=torch.int32,
+                            device="cuda"), n_uniform=64, total_new=64)
+    torch.cuda.synchronize()
+    assert y.yocopp_get_device_status(reset=True) == 0
+    assert_compose_bf16(np_storage(kc)[0, 0].reshape(-1), orc.compose(x1, xi, a1, a2, LAM, "bf16").reshape(-1), orc)
+    assert_compose_bf16(np_storage(vc)[0, 0].reshape(-1), orc.compose(xi, x1, a1, a2, LAM, "bf16").reshape(-1), orc)
