@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--config", type=int, default=3, help="workload (1..5); 3 = 32 x 8192 throughput decode")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the causal prefill-attention measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--decode-kernel", type=int, default=0, choices=[0, 1, 2],
                     help="score product of the decode kernel: 0 default (= 2), 1 CUDA cores, 2 tcgen05 tensor cores")
@@ -82,6 +83,8 @@ KERNEL_SOURCES = {
     "decode_tc_kernel": ["decode_attention_yocopp_b200/csrc/decode_attn_tc.cuh",
                          "decode_attention_yocopp_b200/csrc/decode_attn.cuh",
                          "decode_attention_yocopp_b200/csrc/common.cuh"],
+    "prefill_tc_kernel": ["decode_attention_yocopp_b200/csrc/prefill_attn_tc.cuh",
+                          "decode_attention_yocopp_b200/csrc/common.cuh"],
 }
 
 
@@ -433,6 +436,10 @@ def run_ours(args, rank, world, local):
     t_fused_max = max_over_ranks(fa.elapsed_time(fb), world)
     del step.raw_shared, step.fused_ws
 
+    prefill = None
+    if not args.no_prefill and w.dtype == "bf16" and w.d == 128 and not w.paged:
+        prefill = run_prefill_attention(args, step, world)
+
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, step, world)
@@ -492,6 +499,7 @@ def run_ours(args, rank, world, local):
             "hbm_read_gbs": round(2 * kv_all / (t_fused_max * 1e-3) / 1e9, 1),
             "slowdown_vs_composed_cache": round(t_fused_max / t_attn_max, 3)},
         "roofline": dominant,
+        "prefill_attention": prefill,
         "profiling_trim": bool(args.compose_layers or args.cross_layers),
         "roofline_attention": roof_attn,
         "roofline_compose": roof_comp,
@@ -501,6 +509,63 @@ def run_ours(args, rank, world, local):
         "cpu_baseline": cpu,
     }
     return line
+
+
+def tensor_peak():
+    """Measured dense bf16 tensor throughput (burst, sustained) in TFLOP/s, else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])), "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, 1400.0, "fallback"
+
+
+def causal_pairs(lens) -> int:
+    """(query, key) pairs a whole-prompt causal prefill scores: sum over sequences of n (n + 1) / 2."""
+    return sum(n * (n + 1) // 2 for n in lens)
+
+
+def run_prefill_attention(args, step, world):
+    """Causal prefill attention of the shared self-decoder layer over its own cache
+    (the prefill tokens at positions 0..T-2, already composed by the step), timed
+    per launch with CUDA events.  Algorithmic FLOPs: 4 d (2 for q.k, 2 for p v)
+    per causal (query, key) pair and query head."""
+    import torch
+    import gen
+    w = step.w
+    L = w.shared_layer
+    q = w.device(gen.Q_PREFILL, L)
+    out = torch.empty_like(q)
+    n = w.prefill_lens
+    kw = dict(n_uniform=n[0]) if step.cu is None else dict(cu_q=step.cu, max_q=max(n))
+    for _ in range(2):
+        step.stack.prefill_attend(L, q, out, **kw)
+    torch.cuda.synchronize()
+    K = max(2, min(args.steps, 5))
+    barrier(world)
+    marks = [_event()]
+    for _ in range(K):
+        step.stack.prefill_attend(L, q, out, **kw)
+        marks.append(_event())
+    torch.cuda.synchronize()
+    per = [a.elapsed_time(b) for a, b in zip(marks[:-1], marks[1:])]
+    t_max = max_over_ranks(sum(per), world)
+    flops = 4 * w.d * w.hq * causal_pairs(n)
+    burst, sustained, kind = tensor_peak()
+    ach = flops / (sum(per) / K * 1e-3) / 1e12
+    job = sum_over_ranks(flops * K, world) / (t_max * 1e-3) / 1e12
+    del q, out
+    return {"kernel": "prefill_tc_kernel", "what": "causal attention of one self-decoder layer's prefill tokens "
+                                                   "over its own composed cache (bf16, tcgen05 for q.K and P.V)",
+            "workload": f"{w.name}: {w.batch} x {n[0] if step.cu is None else 'ragged'} prefill tokens, "
+                        f"{w.hq} q / {w.hkv} kv heads, d {w.d}",
+            "launches": K, "ms_per_launch": round(sum(per) / K, 4), "tflops_job": round(job, 1),
+            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": burst, "unit": "TFLOP/s",
+                         "frac": round(ach / burst, 4), "peak_kind": f"{kind} bf16 burst",
+                         "frac_of_sustained": round(ach / sustained, 4),
+                         "algorithmic_flops_per_launch": flops,
+                         "traffic": ncu_traffic("prefill_tc_kernel", w.name)}}
 
 
 def run_e2e(args, step, world):

@@ -30,7 +30,8 @@ YOCOPP_F32 = 1
 EXPORTS = ("yocopp_compose_append", "yocopp_decode_attn_workspace_size", "yocopp_decode_attn",
            "yocopp_get_device_status", "yocopp_status_string", "yocopp_version",
            "yocopp_testing_set_decode_fault", "yocopp_decode_attn_static", "yocopp_decode_attn_partial",
-           "yocopp_decode_combine", "yocopp_decode_attn_fused", "yocopp_set_decode_kernel")
+           "yocopp_decode_combine", "yocopp_decode_attn_fused", "yocopp_set_decode_kernel",
+           "yocopp_prefill_attn")
 
 
 class yocopp_cache(ctypes.Structure):
@@ -86,6 +87,9 @@ def load(path: Optional[str] = None):
     lib.yocopp_decode_combine.argtypes = [V, I32, I64, I32, I32, V, V]
     lib.yocopp_decode_attn_static.restype = I32
     lib.yocopp_decode_attn_static.argtypes = [V, ctypes.POINTER(yocopp_cache), V, V, I32, ctypes.c_float, V]
+    lib.yocopp_prefill_attn.restype = I32
+    lib.yocopp_prefill_attn.argtypes = [V, ctypes.POINTER(yocopp_cache), V, V, I32, I64, I32, V, I32,
+                                        ctypes.c_float, V]
     if path is None:
         _lib = lib
     return lib
@@ -234,6 +238,19 @@ def yocopp_decode_attn_static(q, cache: yocopp_cache, seq_lens, out, num_q_heads
     rc = load().yocopp_decode_attn_static(_ptr(q), ctypes.byref(cache), _ptr(seq_lens), _ptr(out), int(hq),
                                           float(scale), _stream(stream))
     _check("yocopp_decode_attn_static", rc)
+
+
+def yocopp_prefill_attn(q, cache: yocopp_cache, out, pos=None, cu_q=None, n_uniform: int = 0,
+                        total_q: Optional[int] = None, max_q: int = 0, num_q_heads: Optional[int] = None,
+                        scale: float = 0.0, stream=None) -> None:
+    """Causal attention of prefill rows q [total_q][hq][128] (bf16) over the
+    cache's positions [0, pos[b] + j] for row j of sequence b; out like q."""
+    hq = q.shape[1] if num_q_heads is None else num_q_heads
+    if total_q is None:
+        total_q = q.shape[0]
+    rc = load().yocopp_prefill_attn(_ptr(q), ctypes.byref(cache), _ptr(pos), _ptr(cu_q), int(n_uniform),
+                                    int(total_q), int(max_q), _ptr(out), int(hq), float(scale), _stream(stream))
+    _check("yocopp_prefill_attn", rc)
 
 
 STATIC_SCRATCH_BYTES = 4 << 20  # size of the library's fixed scratch array (include/yocopp.h)

@@ -11,6 +11,7 @@
 #include "compose_append.cuh"
 #include "decode_attn.cuh"
 #include "decode_attn_tc.cuh"
+#include "prefill_attn_tc.cuh"
 
 namespace yocopp {
 namespace {
@@ -209,6 +210,45 @@ int32_t launch_decode_tc(const CUtensorMap& tk, const CUtensorMap& tv, const CUt
     lc.attrs = attr;
     lc.numAttrs = 1;
     return cuda_status(cudaLaunchKernelEx(&lc, kern, tk, tv, tq, p));
+}
+
+// ---------------------------------------------------------------- prefill
+// 3-D view of token-major queries [rows][heads][head_dim] (bf16): one box is
+// 64 channels x 1 head x box_rows tokens, 128-byte swizzled.
+bool encode_q3d(CUtensorMap* map, const void* base, int heads, int head_dim, int64_t rows, int box_rows) {
+    EncodeFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[3] = {cuuint64_t(head_dim), cuuint64_t(heads), cuuint64_t(rows)};
+    cuuint64_t gstride[2] = {cuuint64_t(head_dim) * 2, cuuint64_t(heads) * head_dim * 2};
+    cuuint32_t box[3] = {64, 1, cuuint32_t(box_rows)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int32_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p,
+                       int64_t grid, cudaStream_t st) {
+    auto kern = prefill_tc_kernel;
+    static bool attr_set[kMaxDevices] = {false};
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return YOCOPP_ECUDA;
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PfShape::SMEM) != cudaSuccess)
+            return YOCOPP_ECUDA;
+        attr_set[dev] = true;
+    }
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(unsigned(grid), 1, 1);
+    lc.blockDim = dim3(192, 1, 1);
+    lc.dynamicSmemBytes = PfShape::SMEM;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&lc, kern, tq, tk, tv, p));
 }
 
 struct WorkspaceLayout {
@@ -558,5 +598,51 @@ int32_t yocopp_decode_attn_static(const void* q, const yocopp_cache* cache, cons
                               int64_t(kStaticScratchBytes), stream);
 }
 
+// Causal prefill attention of a self-decoder layer over its own cache
+// (tcgen05 for both products).  Argument meaning in yocopp.h.
+int32_t yocopp_prefill_attn(const void* q, const yocopp_cache* cache, const int32_t* pos, const int32_t* cu_q,
+                            int32_t n_uniform, int64_t total_q, int32_t max_q, void* out, int32_t num_q_heads,
+                            float scale, void* stream) {
+    const int32_t rc = check_cache(cache);
+    if (rc != YOCOPP_OK) return rc;
+    if (cache->dtype != YOCOPP_BF16) return YOCOPP_EDTYPE;
+    if (cache->head_dim != 128 || cache->block_table != nullptr) return YOCOPP_EINVAL;
+    if (num_q_heads < 1 || num_q_heads % cache->num_kv_heads != 0) return YOCOPP_EINVAL;
+    if (q == nullptr || out == nullptr || !aligned(q, 16) || !aligned(out, 16)) return YOCOPP_EINVAL;
+    if (!(scale >= 0.f) || !std::isfinite(scale)) return YOCOPP_EINVAL;
+    if (total_q < 0 || total_q >= (int64_t(1) << 31)) return YOCOPP_EINVAL;
+    if (cu_q == nullptr) {
+        if (n_uniform < 0 || int64_t(n_uniform) * cache->batch != total_q) return YOCOPP_EINVAL;
+        max_q = n_uniform;
+    } else if (max_q < 0) {
+        return YOCOPP_EINVAL;
+    }
+    if (int64_t(max_q) > int64_t(cache->capacity)) return YOCOPP_EINVAL;
+    const int64_t rows = int64_t(cache->batch) * cache->num_kv_heads * cache->capacity;
+    if (rows + PfShape::TK >= (int64_t(1) << 31)) return YOCOPP_EINVAL;  // tile row coordinates stay 32-bit
+    if (total_q == 0 || max_q == 0) return YOCOPP_OK;
+    const int q_tiles = (max_q + PfShape::TQ - 1) / PfShape::TQ;
+    const int64_t grid = int64_t(q_tiles) * cache->batch * num_q_heads;
+    if (grid >= (int64_t(1) << 31)) return YOCOPP_EINVAL;
+    alignas(64) CUtensorMap tq, tk, tv;
+    if (!encode_q3d(&tq, q, num_q_heads, 128, total_q, PfShape::TQ) ||
+        !encode_rows(&tk, cache->k, YOCOPP_BF16, 128, rows, PfShape::TK) ||
+        !encode_rows(&tv, cache->v, YOCOPP_BF16, 128, rows, PfShape::TK))
+        return YOCOPP_ECUDA;
+    PrefillParams p;
+    p.out = static_cast<uint8_t*>(out);
+    p.pos = pos;
+    p.cu_q = cu_q;
+    p.n_uniform = cu_q ? 0 : n_uniform;
+    p.batch = cache->batch;
+    p.hq = num_q_heads;
+    p.hkv = cache->num_kv_heads;
+    p.capacity = cache->capacity;
+    p.q_tiles = q_tiles;
+    const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(128.f);
+    p.qscale = sc * 1.4426950408889634f;
+    p.wait_limit_ns = g_wait_limit_ns;
+    return launch_prefill(tq, tk, tv, p, grid, static_cast<cudaStream_t>(stream));
+}
 
 }  // extern "C"

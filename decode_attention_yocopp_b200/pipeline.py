@@ -16,7 +16,7 @@ from typing import Dict, List, Optional, Sequence, Tuple
 
 import torch
 
-from . import (alloc_workspace, make_cache, yocopp_compose_append, yocopp_decode_attn)
+from . import (alloc_workspace, make_cache, yocopp_compose_append, yocopp_decode_attn, yocopp_prefill_attn)
 
 LAMBDA = 35.0
 
@@ -81,3 +81,13 @@ class SharedKVStack:
         yocopp_decode_attn(q, self.desc[i], seq_lens, out, workspace if workspace is not None else self.workspace,
                            self.hq, scale, stream=stream)
         return out
+
+    def prefill_attend(self, i: int, q: torch.Tensor, out: torch.Tensor, pos: Optional[torch.Tensor] = None,
+                       cu_q: Optional[torch.Tensor] = None, n_uniform: int = 0, max_q: int = 0,
+                       scale: float = 0.0, stream=None) -> torch.Tensor:
+        """Self-decoder layer i's causal prefill attention over its own cache, after
+        ``write`` has appended the same tokens (bf16, head_dim 128, contiguous)."""
+        yocopp_prefill_attn(q, self.desc[i], out, pos=pos, cu_q=cu_q, n_uniform=n_uniform, total_q=q.shape[0],
+                            max_q=max_q, num_q_heads=self.hq, scale=scale, stream=stream)
+        return out
+

@@ -33,8 +33,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _HOST_SO = os.path.join(_HERE, "libgen_host.so")
 _DEV_SO = os.path.join(_HERE, "libgen_dev.so")
 
-# tensor kinds (stream ids are kind * 4096 + layer)
-K_PREFILL, V_PREFILL, K_NEW, V_NEW, Q = 1, 2, 3, 4, 5
+# tensor kinds (stream ids are kind * 4096 + layer); Q_PREFILL is the
+# self-decoder layers' queries of the prefill tokens
+K_PREFILL, V_PREFILL, K_NEW, V_NEW, Q, Q_PREFILL = 1, 2, 3, 4, 5, 6
 _SCALARS = 4095  # per-config scalar draws (alpha, lengths, planted position)
 _PERM = 4094     # block-table permutation
 
@@ -230,6 +231,8 @@ class Workload:
             return (self.batch, self.hkv, self.d)
         if kind == Q:
             return (self.batch, self.hq, self.d)
+        if kind == Q_PREFILL:
+            return (self.total_prefill, self.hq, self.d)
         raise ValueError(kind)
 
     def numel(self, kind: int) -> int:

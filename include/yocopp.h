@@ -91,8 +91,10 @@ typedef struct yocopp_cache {
  * computed in fp32 with error-free products and sums for the inner weighted
  * sum (so near-cancelling terms keep their low bits), then multiplied by
  * lambda, rounded once to the cache type, and written to cache positions
- * pos[b] .. pos[b] + n_b - 1.  Stored bf16 values are within one bf16 ulp of
- * the exact composition.
+ * pos[b] .. pos[b] + n_b - 1.  A stored bf16 value is the exact composition
+ * rounded once to nearest-even bf16 (not a rounding of an fp32 intermediate);
+ * only a value within about 2^-48 (relative) of a bf16 rounding midpoint can
+ * land on the other neighbour, so it is always within one bf16 ulp.
  *
  *   K1, V1, Ki, Vi : device, [total_new][num_kv_heads][head_dim], cache dtype,
  *                    16-byte aligned.  Rows are token-major and packed over
@@ -240,6 +242,47 @@ int32_t yocopp_decode_combine(const float* partials, int32_t num_parts, int64_t 
  */
 int32_t yocopp_decode_attn_static(const void* q, const yocopp_cache* cache, const int32_t* seq_lens,
                                   void* out, int32_t num_q_heads, float scale, void* stream);
+
+/*
+ * yocopp_prefill_attn - causal attention of a self-decoder layer's prefill
+ * tokens over that layer's own cache, on the tensor cores (YOCO++: Enhancing
+ * YOCO with KV Residual Connections, section 2 "cache strategy": a lower-half
+ * layer caches its composed K'_i, V'_i and attends over them; section 3:
+ * prefill is compute-bound, the composition adding only a little I/O).
+ * Call it after yocopp_compose_append has written the tokens' composed rows
+ * (the composition and this attention are two kernels in one stream).
+ *
+ * Query row j of sequence b sits at cache position p_b + j (p_b = pos[b], or
+ * 0 when pos == NULL) and, for query head h and KV head g = h / (num_q_heads /
+ * num_kv_heads):
+ *   s_u = scale * <q[b,j,h,:], K'[b,g,u,:]>   for u in [0, p_b + j]
+ *   out[b,j,h,:] = sum_u softmax(s)_u * V'[b,g,u,:]
+ * with fp32 scores and accumulation, P rounded to bf16 for the value product.
+ *
+ *   q       : device bf16 [total_q][num_q_heads][128], 16-byte aligned; rows
+ *             token-major and packed over the batch like yocopp_compose_append's
+ *             inputs: sequence b's rows are [cu_q[b], cu_q[b+1]) or, when
+ *             cu_q == NULL, [b * n_uniform, (b + 1) * n_uniform).
+ *   cache   : HOST descriptor; bf16, head_dim 128, contiguous (block_table
+ *             NULL).  Positions [0, p_b + n_b) of sequence b must hold the
+ *             composed rows.
+ *   pos     : device int32 [batch] or NULL (all 0; a whole-prompt prefill).
+ *   cu_q    : device int32 [batch + 1] prefix offsets, or NULL.
+ *   n_uniform : rows per sequence when cu_q == NULL.
+ *   total_q : rows of q and out (= cu_q[batch] or batch * n_uniform).
+ *   max_q   : with cu_q, an upper bound of every n_b (sizes the grid);
+ *             ignored when cu_q == NULL.
+ *   out     : device bf16 [total_q][num_q_heads][128], 16-byte aligned.
+ *   num_q_heads : multiple of num_kv_heads.
+ *   scale   : softmax scale; 0 selects 1/sqrt(128).
+ * A sequence with p_b < 0, p_b + n_b > capacity or n_b > max_q is skipped and
+ * YOCOPP_ECAPACITY recorded on the device; a decreasing cu_q records
+ * YOCOPP_EDEVICE_CHECK.  Output rows of skipped sequences are not written.
+ * Returns YOCOPP_EDTYPE for fp32 caches and YOCOPP_EINVAL for other shapes.
+ */
+int32_t yocopp_prefill_attn(const void* q, const yocopp_cache* cache, const int32_t* pos, const int32_t* cu_q,
+                            int32_t n_uniform, int64_t total_q, int32_t max_q, void* out, int32_t num_q_heads,
+                            float scale, void* stream);
 
 /*
  * yocopp_get_device_status - the first error code recorded by a kernel on

@@ -57,6 +57,7 @@ def load(path: Optional[str] = None):
     lib.orc_attention_partial.argtypes = [P, P, P, I, I64, I64, I, I, D, P, P, P, P]
     lib.orc_lse_combine.argtypes = [I, P, P, P, I, I, P]
     lib.orc_attention.argtypes = [P, P, P, I, I64, I, I, D, P, P, P]
+    lib.orc_causal_attention.argtypes = [P, P, P, I, I64, I64, I, D, P, P]
     return lib
 
 
@@ -118,6 +119,22 @@ class Oracle:
         self.lib.orc_attention(q.ctypes.data, K.ctypes.data, V.ctypes.data, _DT[dtype], n, d, G, scale,
                                scores.ctypes.data, out.ctypes.data, w.ctypes.data if weights else None)
         return (out, w[:, :n]) if weights else out
+
+    def causal_attention(self, q: np.ndarray, K: np.ndarray, V: np.ndarray, dtype: str, scale: float,
+                         p0: int = 0) -> np.ndarray:
+        """Causal attention of query rows q [n][d] (fp64) sitting at cache positions
+        p0 .. p0 + n - 1 over K, V [len][d] (storage form, len >= p0 + n): row j
+        attends to positions 0 .. p0 + j.  Returns [n][d] fp64."""
+        q = np.ascontiguousarray(q, dtype=np.float64)
+        n, d = q.shape
+        K = np.ascontiguousarray(K, dtype=_NP[dtype]).reshape(-1, d)
+        V = np.ascontiguousarray(V, dtype=_NP[dtype]).reshape(-1, d)
+        assert K.shape[0] == V.shape[0] >= p0 + n and p0 >= 0
+        scores = np.empty(max(1, p0 + n), dtype=np.float64)
+        out = np.empty((n, d), dtype=np.float64)
+        self.lib.orc_causal_attention(q.ctypes.data, K.ctypes.data, V.ctypes.data, _DT[dtype], int(p0), n, d,
+                                      scale, scores.ctypes.data, out.ctypes.data)
+        return out
 
     def attention_partial(self, q, K, V, dtype: str, t0: int, t1: int, scale: float):
         q = np.ascontiguousarray(q, dtype=np.float64)

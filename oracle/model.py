@@ -84,3 +84,39 @@ def decode_self_group(orc: Oracle, w: "gen.Workload", layer: int, b: int, g: int
         K, V = kv
     q = query(w, layer, b)[g * w.group:(g + 1) * w.group]
     return orc.attention(q, K, V, w.dtype, default_scale(w.d) if scale is None else scale)
+
+
+def prefill_queries(w: "gen.Workload", layer: int, b: int, rows: np.ndarray) -> np.ndarray:
+    """Prefill queries of self-decoder ``layer`` for sequence b at the given token
+    positions (0 .. T-2): [len(rows)][Hq][d] fp64 (exact)."""
+    rows = np.asarray(rows, dtype=np.int64)
+    if rows.size == 0:
+        return np.zeros((0, w.hq, w.d), dtype=np.float64)
+    lo, hi = int(rows.min()), int(rows.max()) + 1
+    base = int(w.cu_prefill[b])
+    if hi - lo <= 4 * rows.size:  # dense: one span
+        block = w.host_rows(gen.Q_PREFILL, layer, base + lo, hi - lo)
+        return storage_to_f64(block[rows - lo], w.dtype)
+    return storage_to_f64(np.stack([w.host_rows(gen.Q_PREFILL, layer, base + int(t), 1)[0] for t in rows]), w.dtype)
+
+
+def prefill_self_rows(orc: Oracle, w: "gen.Workload", layer: int, b: int, h: int, rows,
+                      kv: Tuple[np.ndarray, np.ndarray] | None = None, scale: float | None = None) -> np.ndarray:
+    """Self-decoder layer ``layer`` during prefill (YOCO++ section 2, cache strategy;
+    section 3, prefill): prefill token t of sequence b, query head h, attends
+    causally over cache positions 0..t of its layer's stored cache (KV head
+    h // group).  Returns [len(rows)][d] fp64 for the requested token positions."""
+    g = h // w.group
+    if kv is None:
+        K = composed_seq(orc, w, layer, "K", b, g)
+        V = composed_seq(orc, w, layer, "V", b, g)
+    else:
+        K, V = kv
+    rows = np.asarray(rows, dtype=np.int64)
+    q = prefill_queries(w, layer, b, rows)[:, h, :]
+    sc = default_scale(w.d) if scale is None else scale
+    out = np.empty((rows.size, w.d), dtype=np.float64)
+    for i, t in enumerate(rows):
+        out[i] = orc.causal_attention(q[i:i + 1], K, V, w.dtype, sc, p0=int(t))[0]
+    return out
+

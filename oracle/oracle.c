@@ -21,6 +21,13 @@
  *                    sum_t p_t V_t, written as the textbook two-pass softmax
  *                    (max, then exponentials and their sum).  A one-token
  *                    query needs no causal mask inside the cache.
+ *   orc_causal_attention
+ *                    a self-decoder layer's prefill attention over the cache
+ *                    it stores (YOCO++: Enhancing YOCO with KV Residual
+ *                    Connections, section 2, cache strategy; section 3,
+ *                    prefill): a token at cache position t attends causally
+ *                    to positions 0..t, i.e. orc_attention of its query over
+ *                    the first t + 1 cached rows.
  *   orc_attention_partial / orc_lse_combine
  *                    the same attention restricted to a token range, kept
  *                    unnormalised as (max, sum of exponentials, weighted sum),
@@ -170,5 +177,20 @@ void orc_attention(const double* q, const void* K, const void* V, int dtype, int
             if (weights) weights[(int64_t)h * len + t] = p;
             for (int c = 0; c < d; ++c) oh[c] += p * load(V, dtype, t * d + c);
         }
+    }
+}
+
+/*
+ * Causal attention of a chunk of n query rows over a layer's own cache.
+ * Row j of q [n][d] (fp64) is the token at cache position p0 + j; it attends
+ * to cache positions 0 .. p0 + j of K/V [len][d] (len >= p0 + n), so its
+ * output is the one-query orc_attention over the first p0 + j + 1 rows.
+ *   scores: scratch of at least p0 + n doubles;  out [n][d] fp64.
+ */
+void orc_causal_attention(const double* q, const void* K, const void* V, int dtype, int64_t p0, int64_t n,
+                          int d, double scale, double* scores, double* out) {
+    for (int64_t j = 0; j < n; ++j) {
+        const int64_t visible = p0 + j + 1;
+        orc_attention(q + j * d, K, V, dtype, visible, d, 1, scale, scores, out + j * d, NULL);
     }
 }

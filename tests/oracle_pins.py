@@ -296,4 +296,91 @@ def pin_planted_key(orc):
     assert np.max(np.abs(got[0] - V[p])) <= max(bound, 1e-12)
 
 
+# ---------------------------------------------------------------------------
+# causal prefill attention (YOCO++ section 2, cache strategy: each self-decoder
+# layer attends over the composed KV set it stores; a token sees positions
+# up to its own)
+# ---------------------------------------------------------------------------
+
+def pin_causal_first_row(orc):
+    """A whole-prompt chunk (p0 = 0): the first token sees only itself, so its
+    output is its own value row, exactly."""
+    rng = _rng(20)
+    for dtype in ("bf16", "f32"):
+        if dtype == "bf16":
+            K, V = _rand_bf16(rng, (9, 32)), _rand_bf16(rng, (9, 32))
+            v0 = _f64(V[0])
+        else:
+            K = rng.standard_normal((9, 32)).astype(np.float32)
+            V = rng.standard_normal((9, 32)).astype(np.float32)
+            v0 = V[0].astype(np.float64)
+        got = orc.causal_attention(rng.standard_normal((9, 32)) * 4, K, V, dtype, 0.2)
+        assert np.array_equal(got[0], v0)
+
+
+def pin_causal_identical_keys(orc):
+    """Identical keys: row j weighs positions 0..p0+j equally, so it is the mean
+    of the first p0 + j + 1 value rows (also with earlier context, p0 > 0)."""
+    rng = _rng(21)
+    n, d = 23, 16
+    for p0 in (0, 1, 7):
+        K = np.tile(rng.standard_normal(d), (p0 + n + 3, 1))
+        V = rng.standard_normal((p0 + n + 3, d))
+        got = orc.causal_attention(rng.standard_normal((n, d)), K, V, "f64", 0.3, p0=p0)
+        want = np.stack([V[:p0 + j + 1].mean(axis=0) for j in range(n)])
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def pin_causal_query_row(orc):
+    """One-hot keys and queries: row j's query matches only the key at its own
+    position p0 + j, so the output is (to e^-36) that position's value row."""
+    rng = _rng(22)
+    p0, n, d = 4, 12, 16
+    K = 6.0 * np.eye(d)
+    V = rng.standard_normal((d, d))
+    q = np.stack([6.0 * np.eye(d)[p0 + j] for j in range(n)])
+    got = orc.causal_attention(q, K, V, "f64", 1.0, p0=p0)
+    np.testing.assert_allclose(got, V[p0:p0 + n], rtol=0, atol=1e-12)
+
+
+def pin_causal_future_invariance(orc):
+    """Row j ignores every position after p0 + j and depends on position p0 + j."""
+    rng = _rng(23)
+    p0, n, d = 3, 40, 16
+    K = rng.standard_normal((p0 + n, d)) * 2
+    V = rng.standard_normal((p0 + n, d))
+    q = rng.standard_normal((n, d))
+    base = orc.causal_attention(q, K, V, "f64", 0.4, p0=p0)
+    j = 17
+    K2, V2 = K.copy(), V.copy()
+    K2[p0 + j + 1:] = rng.standard_normal(K2[p0 + j + 1:].shape) * 5
+    V2[p0 + j + 1:] += 3.0
+    got = orc.causal_attention(q, K2, V2, "f64", 0.4, p0=p0)
+    np.testing.assert_array_equal(got[:j + 1], base[:j + 1])
+    assert np.min(np.max(np.abs(got[j + 1:] - base[j + 1:]), axis=1)) > 1e-6
+    V3 = V.copy()
+    V3[p0 + j] += 1.0
+    assert np.max(np.abs(orc.causal_attention(q, K, V3, "f64", 0.4, p0=p0)[j] - base[j])) > 1e-6
+
+
+def pin_causal_matches_sdpa(orc):
+    """Library special case: torch's fp64 CPU scaled_dot_product_attention with
+    the causal mask (is_causal for p0 = 0, an explicit boolean mask otherwise)."""
+    import torch
+    rng = _rng(24)
+    for p0, n, d in ((0, 130, 64), (0, 257, 128), (100, 77, 128)):
+        K = rng.standard_normal((p0 + n, d)) * 2
+        V = rng.standard_normal((p0 + n, d))
+        q = rng.standard_normal((n, d))
+        scale = 1.0 / math.sqrt(d)
+        got = orc.causal_attention(q, K, V, "f64", scale, p0=p0)
+        tq, tk, tv = (torch.from_numpy(x)[None, None] for x in (q, K, V))
+        if p0 == 0:
+            ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True, scale=scale)
+        else:
+            mask = torch.arange(p0 + n)[None, :] <= (p0 + torch.arange(n))[:, None]
+            ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=scale)
+        np.testing.assert_allclose(got, ref[0, 0].numpy(), rtol=0, atol=1e-12)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

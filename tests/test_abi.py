@@ -84,3 +84,26 @@ def test_decode_kernel_selector():
         assert lib.yocopp_set_decode_kernel(which) == y.YOCOPP_OK
     assert lib.yocopp_set_decode_kernel(3) == y.YOCOPP_EINVAL
     assert lib.yocopp_set_decode_kernel(-1) == y.YOCOPP_EINVAL
+
+
+def test_prefill_host_checks():
+    lib = y.load()
+    c = _cache()
+    # shapes the tensor-core prefill does not take
+    assert lib.yocopp_prefill_attn(0x10, ctypes.byref(_cache(dtype=y.YOCOPP_F32)), None, None, 4, 8, 0, 0x10, 32, 0.0,
+                                   None) == y.YOCOPP_EDTYPE
+    assert lib.yocopp_prefill_attn(0x10, ctypes.byref(_cache(head_dim=64)), None, None, 4, 8, 0, 0x10, 32, 0.0,
+                                   None) == y.YOCOPP_EINVAL
+    paged = _cache(block_table=0x3000, block_size=64, max_blocks_per_seq=1, num_blocks=4)
+    assert lib.yocopp_prefill_attn(0x10, ctypes.byref(paged), None, None, 4, 8, 0, 0x10, 32, 0.0, None) == y.YOCOPP_EINVAL
+    # query heads, pointers, alignment, scale, counts
+    assert lib.yocopp_prefill_attn(0x10, ctypes.byref(c), None, None, 4, 8, 0, 0x10, 12, 0.0, None) == y.YOCOPP_EINVAL
+    assert lib.yocopp_prefill_attn(None, ctypes.byref(c), None, None, 4, 8, 0, 0x10, 32, 0.0, None) == y.YOCOPP_EINVAL
+    assert lib.yocopp_prefill_attn(0x18, ctypes.byref(c), None, None, 4, 8, 0, 0x10, 32, 0.0, None) == y.YOCOPP_EINVAL
+    assert lib.yocopp_prefill_attn(0x10, ctypes.byref(c), None, None, 4, 8, 0, 0x10, 32, -1.0, None) == y.YOCOPP_EINVAL
+    assert lib.yocopp_prefill_attn(0x10, ctypes.byref(c), None, None, 4, 9, 0, 0x10, 32, 0.0, None) == y.YOCOPP_EINVAL
+    assert lib.yocopp_prefill_attn(0x10, ctypes.byref(c), None, None, 65, 130, 0, 0x10, 32, 0.0, None) == y.YOCOPP_EINVAL
+    assert lib.yocopp_prefill_attn(0x10, ctypes.byref(c), None, 0x20, 0, 8, -1, 0x10, 32, 0.0, None) == y.YOCOPP_EINVAL
+    assert lib.yocopp_prefill_attn(0x10, ctypes.byref(c), None, 0x20, 0, 8, 65, 0x10, 32, 0.0, None) == y.YOCOPP_EINVAL
+    # nothing to do is a no-op success
+    assert lib.yocopp_prefill_attn(0x10, ctypes.byref(c), None, None, 0, 0, 0, 0x10, 32, 0.0, None) == y.YOCOPP_OK

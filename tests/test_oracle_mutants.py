@@ -34,6 +34,10 @@ MUTANTS = {
     "combine_no_divide": ("for (int c = 0; c < d; ++c) oh[c] /= L;", ""),
     "partial_wrong_max": ("if (s > mx) mx = s;", "if (s < mx) mx = s;"),
     "head_stride": ("const double* qh = q + (int64_t)h * d;\n        double* oh", "const double* qh = q;\n        double* oh"),
+    "causal_excludes_self": ("const int64_t visible = p0 + j + 1;", "const int64_t visible = p0 + j;"),
+    "causal_ignores_offset": ("const int64_t visible = p0 + j + 1;", "const int64_t visible = j + 1;"),
+    "causal_whole_chunk": ("const int64_t visible = p0 + j + 1;", "const int64_t visible = p0 + n;"),
+    "causal_first_query": ("orc_attention(q + j * d, K, V", "orc_attention(q, K, V"),
 }
 
 
