@@ -10,26 +10,36 @@
 // cache positions [0, p_b + j] of KV head g = h / (hq / hkv):
 //   out[b,j,h] = sum_u softmax_u(scale q . K'_u) V'_u.
 //
-// One CTA per (sequence, query head, 128-row query tile), heaviest query
-// tiles first.  Tensor memory holds S (128 x 128 fp32, columns 0..127) and
-// the output accumulator O (128 x 128 fp32, columns 128..255).  Per key tile:
-//   S = Q K^T   eight tcgen05.mma (M = 128 queries, N = 128 keys, K = 16
-//               channels each), Q and K K-major straight from their TMA tiles;
-//   softmax     one thread per query row reads its S row, masks keys past
-//               its position, and forms P = 2^(s - m) against a reference
-//               maximum m that moves only when the row maximum exceeds it by
-//               more than 8 (then O and the row sum are rescaled), so P <= 2^8
-//               and the rescale is rare; P goes to shared memory as bf16 in
-//               the 128-byte swizzled K-major layout the MMA reads;
-//   O += P V    eight tcgen05.mma (M = 128, N = 128 channels, K = 16 keys)
-//               with V read MN-major from its TMA tile.
-// The next tile's S product is issued before this tile's P V so that the
-// tensor cores work while the softmax threads do.
+// Work unit: one CTA per (sequence, 128-row query tile, pair of query heads
+// of one KV head), heaviest query tiles first.  The two heads ("a" and "b")
+// share every K/V tile the CTA loads, which halves the K/V traffic per FLOP
+// (a lone head per CTA streams 64 KB of K/V per 8.4 MFLOP, more than L2 can
+// feed every SM at tensor-core speed).  With an odd group size each CTA takes
+// one head.
 //
-// Warps: 0 = TMA producer, 1 = MMA issuer and tensor-memory owner, 2..5 =
-// softmax and epilogue (warp w reads TMEM lanes 32 (w mod 4) .. + 31).  Every
-// wait is bounded; on a timeout the kernel records YOCOPP_ETIMEOUT, waits
-// (bounded) for its own copies in flight, frees the tensor memory and returns.
+// Tensor memory (512 columns): S_a, S_b (128 x 128 fp32 each) and O_a, O_b.
+// Per key tile t and head x:
+//   S_x = Q_x K^T  eight tcgen05.mma (M = 128 queries, N = 128 keys, K = 16
+//                  channels), Q and K K-major from their TMA tiles;
+//   softmax        one thread per query row: masks keys past its position,
+//                  forms P = 2^(s - m) against a reference maximum m that
+//                  moves only when the row maximum exceeds it by more than 8
+//                  (then O_x and the row sum are rescaled), so P <= 2^8 and
+//                  rescales are rare; P is written as bf16 into the first 64
+//                  columns of S_x (two keys per column), where the next
+//                  product reads it;
+//   O_x += P V     eight tcgen05.mma (M = 128, N = 128 channels, K = 16 keys)
+//                  with P from tensor memory and V MN-major from its TMA tile.
+// The tensor pipe runs PV_a(t), QK_a(t+1), PV_b(t), QK_b(t+1): while one
+// head's softmax works, the other head's products run.  K and V stream
+// through separate two-slot rings, each refilled by its own producer lane as
+// soon as the last product reading the slot completes.
+//
+// Warps: 0 = TMA producer (lane 0: Q and K, lane 1: V), 1 = MMA issuer and
+// tensor-memory owner, 2..5 = softmax and epilogue of head a, 6..9 = head b
+// (warp w reads TMEM lanes 32 (w mod 4) .. + 31).  Every wait is bounded; on
+// a timeout the kernel records YOCOPP_ETIMEOUT, waits (bounded) for its own
+// copies and products in flight, frees the tensor memory and returns.
 #pragma once
 
 #include "decode_attn.cuh"
@@ -43,6 +53,7 @@ struct PrefillParams {
     int32_t n_uniform;
     int32_t batch, hq, hkv, capacity;
     int32_t q_tiles;        // ceil(max query rows per sequence / 128)
+    int32_t heads_per_cta;  // 2 (group size even) or 1
     float qscale;           // softmax scale * log2(e)
     uint64_t wait_limit_ns;
 };
@@ -51,19 +62,42 @@ struct PfShape {
     static constexpr int D = 128, TQ = 128, TK = 128;
     static constexpr int BOXB = 128 * 128;          // one [128 rows][128 B] swizzled box
     static constexpr int TILE_BYTES = 2 * BOXB;     // 128 rows x 128 channels, bf16
-    static constexpr int Q_OFF = 0;
-    static constexpr int KV_OFF = TILE_BYTES;       // 2 stages x (K tile, V tile)
-    static constexpr int P_OFF = KV_OFF + 4 * TILE_BYTES;
-    static constexpr int BAR_OFF = P_OFF + TILE_BYTES;
-    static constexpr int NBAR = 9;                  // q_full, kv_full[2], kv_empty[2], s_full, s_free, p_full, o_done
+    static constexpr int KSLOTS = 2, VSLOTS = 2;
+    static constexpr int Q_OFF = 0;                 // Q_a, Q_b
+    static constexpr int K_OFF = 2 * TILE_BYTES;
+    static constexpr int V_OFF = K_OFF + KSLOTS * TILE_BYTES;
+    static constexpr int BAR_OFF = V_OFF + VSLOTS * TILE_BYTES;
+    // q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2], o_done[2], drain
+    static constexpr int NBAR = 16;
     static constexpr int SMEM = 1024 + BAR_OFF + NBAR * 8 + 16;
+    static constexpr int THREADS = 320;
     static constexpr uint32_t IDESC_QK = umma_idesc_bf16(128, 128, false);
     static constexpr uint32_t IDESC_PV = umma_idesc_bf16(128, 128, true);
-    static constexpr int TMEM_COLS = 256;
+    static constexpr int TMEM_COLS = 512;           // S_a 0, S_b 128, O_a 256, O_b 384
     static constexpr float RESCALE_SLACK = 8.f;     // log2 of the largest P before a rescale
 };
+static_assert(PfShape::SMEM <= 232448 - 16, "prefill shared memory");
 
-__global__ void __launch_bounds__(192, 1)
+// 2^x on the FMA pipe, for x <= 2^22 (x below -126 is taken as -126, whose
+// result, at most 2^-125.5, is nothing next to the row's largest term 1):
+// x = j + f with j = round(x), f in [-1/2, 1/2] (Cody and Waite's range
+// reduction, with the round done by adding 1.5 * 2^23), 2^f from a cubic
+// fitted here to the relative error on [-1/2, 1/2] (max 7.5e-5, far below
+// the 2^-9 of the bf16 probabilities it feeds), and 2^j added to the exponent
+// field.  The exponential unit does 16 results per clock per SM, one tile's
+// worth in the time the tensor cores take for it; moving a quarter of them
+// here keeps it off the critical path.
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -126.f);  // keeps the exponent field of the result >= 0
+    const float t = x + 12582912.f;          // 1.5 * 2^23: round to integer in the low mantissa bits
+    const float f = x - (t - 12582912.f);
+    float p = fmaf(0x1.c3f76p-5f, f, 0x1.f0de1ap-3f);
+    p = fmaf(p, f, 0x1.62f31ap-1f);
+    p = fmaf(p, f, 0x1.fff692p-1f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+__global__ void __launch_bounds__(PfShape::THREADS, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
     using S = PfShape;
@@ -73,11 +107,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 
     griddep_wait();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int per_tile = p.batch * p.hq;
-    const int jt = p.q_tiles - 1 - int(blockIdx.x) / per_tile;  // heaviest (latest) query tiles first
+    const int G = p.hq / p.hkv;
+    const int units = G / p.heads_per_cta;                         // CTAs per (sequence, KV head, tile)
+    const int per_tile = p.batch * p.hkv * units;
+    const int jt = p.q_tiles - 1 - int(blockIdx.x) / per_tile;     // heaviest (latest) query tiles first
     const int rem = int(blockIdx.x) % per_tile;
-    const int b = rem / p.hq, h = rem % p.hq;
-    const int g = h / (p.hq / p.hkv);
+    const int b = rem / (p.hkv * units);
+    const int g = (rem / units) % p.hkv;
+    const int h0 = g * G + (rem % units) * p.heads_per_cta;
+    const bool pair = p.heads_per_cta == 2;
+    const int nsm = pair ? 8 : 4;                                  // softmax warps in use
     int qrow0, nq;
     if (p.cu_q) {
         qrow0 = __ldg(p.cu_q + b);
@@ -88,11 +127,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     }
     const int p0 = p.pos ? __ldg(p.pos + b) : 0;
     if (nq < 0) {
-        if (tid == 0 && jt == 0 && h == 0) record_status(YOCOPP_EDEVICE_CHECK);
+        if (tid == 0 && jt == 0 && rem % (p.hkv * units) == 0) record_status(YOCOPP_EDEVICE_CHECK);
         return;
     }
     if (p0 < 0 || int64_t(p0) + nq > p.capacity || nq > p.q_tiles * S::TQ) {
-        if (tid == 0 && jt == 0 && h == 0) record_status(YOCOPP_ECAPACITY);
+        if (tid == 0 && jt == 0 && rem % (p.hkv * units) == 0) record_status(YOCOPP_ECAPACITY);
         return;
     }
     if (jt * S::TQ >= nq) return;
@@ -102,28 +141,30 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const int qpos_first = p0 + jt * S::TQ;          // smallest query position in the tile
 
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* Qs = base + S::Q_OFF;
-    uint8_t* Ps = base + S::P_OFF;
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + S::BAR_OFF);
     uint64_t* q_full = bars + 0;
-    uint64_t* kv_full = bars + 1;   // [2]
-    uint64_t* kv_empty = bars + 3;  // [2]
-    uint64_t* s_full = bars + 5;
-    uint64_t* s_free = bars + 6;
-    uint64_t* p_full = bars + 7;
-    uint64_t* o_done = bars + 8;
+    uint64_t* k_full = bars + 1;    // [2]
+    uint64_t* k_empty = bars + 3;   // [2]
+    uint64_t* v_full = bars + 5;    // [2]
+    uint64_t* v_empty = bars + 7;   // [2]
+    uint64_t* s_full = bars + 9;    // [head]
+    uint64_t* p_full = bars + 11;   // [head]
+    uint64_t* o_done = bars + 13;   // [head]
+    uint64_t* drain = bars + 15;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + S::BAR_OFF + S::NBAR * 8);
 
     if (tid == 0) {
         mbar_init(q_full, 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+            mbar_init(&s_full[s], 1);
+            mbar_init(&p_full[s], 4);
+            mbar_init(&o_done[s], 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(s_free, 4);
-        mbar_init(p_full, 4);
-        mbar_init(o_done, 1);
+        mbar_init(drain, 1);
         fence_mbar_init();
         s_abort = 0;
         s_cdone = 0;
@@ -136,35 +177,38 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tO = tmem + 128;
 
     if (warp == 0) {
-        // ------------------------------------------------------------------ producer
-        if (lane == 0) {
-            int last_t[2] = {-1, -1};
+        // ------------------------------------------------------------------ producers
+        if (lane < 2) {
+            const bool kl = lane == 0;   // lane 0: Q and the K ring; lane 1: the V ring
+            const CUtensorMap* map = kl ? &tmK : &tmV;
+            uint64_t* full = kl ? k_full : v_full;
+            uint64_t* empty = kl ? k_empty : v_empty;
+            uint8_t* ring = base + (kl ? S::K_OFF : S::V_OFF);
+            int issued = 0;
             bool ok = true;
-            prefetch_tensormap(&tmQ);
-            prefetch_tensormap(&tmK);
-            prefetch_tensormap(&tmV);
-            mbar_arrive_expect_tx(q_full, uint32_t(S::TILE_BYTES));
-            for (int bx = 0; bx < 2; ++bx)
-                tma_load_3d(Qs + bx * S::BOXB, &tmQ, q_full, bx * 64, h, qrow0 + jt * S::TQ);
+            prefetch_tensormap(map);
+            if (kl) {
+                prefetch_tensormap(&tmQ);
+                mbar_arrive_expect_tx(q_full, uint32_t((pair ? 2 : 1) * S::TILE_BYTES));
+                for (int x = 0; x < (pair ? 2 : 1); ++x)
+                    for (int bx = 0; bx < 2; ++bx)
+                        tma_load_3d(base + S::Q_OFF + x * S::TILE_BYTES + bx * S::BOXB, &tmQ, q_full, bx * 64,
+                                    h0 + x, qrow0 + jt * S::TQ);
+            }
             const int plane_row = (b * p.hkv + g) * p.capacity;
             for (int t = 0; t < ntk; ++t) {
-                const int st = t & 1;
-                if (s_abort || !mbar_wait(&kv_empty[st], ((t >> 1) & 1) ^ 1, p.wait_limit_ns)) {
+                const int slot = t & 1;
+                if (s_abort || !mbar_wait(&empty[slot], ((t >> 1) & 1) ^ 1, p.wait_limit_ns)) {
                     ok = false;
                     break;
                 }
-                uint8_t* ks = base + S::KV_OFF + st * 2 * S::TILE_BYTES;
-                uint8_t* vs = ks + S::TILE_BYTES;
-                mbar_arrive_expect_tx(&kv_full[st], uint32_t(2 * S::TILE_BYTES));
-                const int row = plane_row + t * S::TK;
-                for (int bx = 0; bx < 2; ++bx) {
-                    tma_load_2d(ks + bx * S::BOXB, &tmK, &kv_full[st], bx * 64, row);
-                    tma_load_2d(vs + bx * S::BOXB, &tmV, &kv_full[st], bx * 64, row);
-                }
-                last_t[st] = t;
+                mbar_arrive_expect_tx(&full[slot], uint32_t(S::TILE_BYTES));
+                for (int bx = 0; bx < 2; ++bx)
+                    tma_load_2d(ring + slot * S::TILE_BYTES + bx * S::BOXB, map, &full[slot], bx * 64,
+                                plane_row + t * S::TK);
+                issued = t + 1;
             }
             if (!ok) {
                 record_status(YOCOPP_ETIMEOUT);
@@ -172,9 +216,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             }
             if (!ok || s_abort) {
                 // let the copies this thread issued land before the CTA can exit
-                (void)mbar_wait(q_full, 0, p.wait_limit_ns);
-                for (int st = 0; st < 2; ++st)
-                    if (last_t[st] >= 0) (void)mbar_wait(&kv_full[st], (last_t[st] >> 1) & 1, p.wait_limit_ns);
+                if (kl) (void)mbar_wait(q_full, 0, p.wait_limit_ns);
+                for (int t = issued > 2 ? issued - 2 : 0; t < issued; ++t)
+                    (void)mbar_wait(&full[t & 1], (t >> 1) & 1, p.wait_limit_ns);
             }
         }
         return;
@@ -183,57 +227,81 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     if (warp == 1) {
         // ------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t qaddr = smem_addr(Qs);
-            const uint32_t paddr = smem_addr(Ps);
-            const uint32_t kvaddr = smem_addr(base + S::KV_OFF);
+            const uint32_t qaddr = smem_addr(base + S::Q_OFF);
+            const uint32_t kaddr0 = smem_addr(base + S::K_OFF);
+            const uint32_t vaddr0 = smem_addr(base + S::V_OFF);
             bool ok = mbar_wait(q_full, 0, p.wait_limit_ns);
-            int pv_issued = 0;
-            auto issue_qk = [&](int t) -> bool {
-                if (s_abort || !mbar_wait(&kv_full[t & 1], (t >> 1) & 1, p.wait_limit_ns) ||
-                    !mbar_wait(s_free, (t & 1) ^ 1, p.wait_limit_ns))
-                    return false;
-                tc_fence_after();
-                const uint32_t kaddr = kvaddr + uint32_t((t & 1) * 2 * S::TILE_BYTES);
+            bool issued_any = false;
+            auto qk = [&](int x, int t) {
+                const uint32_t ka = kaddr0 + uint32_t((t & 1) * S::TILE_BYTES);
+                const uint32_t qa = qaddr + uint32_t(x * S::TILE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < S::D / 16; ++kk) {
                     const uint32_t off = uint32_t((kk >> 2) * S::BOXB + (kk & 3) * 32);
-                    umma_bf16(tS, umma_desc_sw128(qaddr + off), umma_desc_sw128(kaddr + off), S::IDESC_QK,
+                    umma_bf16(tmem + 128 * x, umma_desc_sw128(qa + off), umma_desc_sw128(ka + off), S::IDESC_QK,
                               kk > 0 ? 1u : 0u);
                 }
-                umma_commit(s_full);
-                return true;
+                umma_commit(&s_full[x]);
+                issued_any = true;
             };
-            if (ok) ok = issue_qk(0);
+            auto pv = [&](int x, int t) {
+                const uint32_t va = vaddr0 + uint32_t((t & 1) * S::TILE_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < S::TK / 16; ++kk)
+                    umma_bf16_tmem_a(tmem + 256 + 128 * x, tmem + 128 * x + 8 * kk,
+                                     umma_desc_sw128_mn(va + uint32_t(kk * 16 * 128), S::BOXB, 1024), S::IDESC_PV,
+                                     (t > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&o_done[x]);
+                issued_any = true;
+            };
+            if (ok) ok = !s_abort && mbar_wait(&k_full[0], 0, p.wait_limit_ns);
+            if (ok) {
+                tc_fence_after();
+                qk(0, 0);
+                if (pair) qk(1, 0);
+                umma_commit(&k_empty[0]);
+            }
             for (int t = 0; ok && t < ntk; ++t) {
-                if (t + 1 < ntk && !issue_qk(t + 1)) {
-                    ok = false;
-                    break;
-                }
-                if (s_abort || !mbar_wait(p_full, t & 1, p.wait_limit_ns)) {
+                const bool more = t + 1 < ntk;
+                // head a: P V of tile t, then S of tile t + 1
+                if (s_abort || !mbar_wait(&p_full[0], t & 1, p.wait_limit_ns) ||
+                    !mbar_wait(&v_full[t & 1], (t >> 1) & 1, p.wait_limit_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t vaddr = kvaddr + uint32_t((t & 1) * 2 * S::TILE_BYTES + S::TILE_BYTES);
-#pragma unroll
-                for (int kk = 0; kk < S::TK / 16; ++kk) {
-                    const uint32_t aoff = uint32_t((kk >> 2) * S::BOXB + (kk & 3) * 32);
-                    umma_bf16(tO, umma_desc_sw128(paddr + aoff),
-                              umma_desc_sw128_mn(vaddr + uint32_t(kk * 16 * 128), S::BOXB, 1024), S::IDESC_PV,
-                              (t > 0 || kk > 0) ? 1u : 0u);
+                pv(0, t);
+                if (more) {
+                    if (!mbar_wait(&k_full[(t + 1) & 1], ((t + 1) >> 1) & 1, p.wait_limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    qk(0, t + 1);
                 }
-                umma_commit(o_done);
-                umma_commit(&kv_empty[t & 1]);
-                pv_issued = t + 1;
+                if (pair) {
+                    if (s_abort || !mbar_wait(&p_full[1], t & 1, p.wait_limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    pv(1, t);
+                    if (more) qk(1, t + 1);
+                }
+                umma_commit(&v_empty[t & 1]);
+                if (more) umma_commit(&k_empty[(t + 1) & 1]);
             }
             if (!ok) {
                 record_status(YOCOPP_ETIMEOUT);
                 s_abort = 1;
+                if (issued_any) {  // every product issued finishes before the tensor memory is freed
+                    umma_commit(drain);
+                    (void)mbar_wait(drain, 0, p.wait_limit_ns);
+                }
             }
             // the softmax warps finish reading O before the tensor memory is freed
             const uint64_t t0 = globaltimer_ns();
-            while (atomicAdd(&s_cdone, 0) < 4 && globaltimer_ns() - t0 <= p.wait_limit_ns) __nanosleep(256);
-            if (!ok && pv_issued > 0) (void)mbar_wait(o_done, (pv_issued - 1) & 1, p.wait_limit_ns);
+            while (atomicAdd(&s_cdone, 0) < nsm && globaltimer_ns() - t0 <= p.wait_limit_ns) __nanosleep(256);
         }
         __syncwarp();
         tc_fence_after();
@@ -242,40 +310,38 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     }
 
     // ------------------------------------------------------------ softmax + epilogue
+    const int x = (warp - 2) >> 2;                  // head of this warpgroup (0 = a, 1 = b)
+    if (x == 1 && !pair) return;
     const int qd = warp & 3;
     const int r = 32 * qd + lane;                   // query row in the tile (TMEM lane)
     const int j = jt * S::TQ + r;                   // query row in the sequence
     const int qpos = p0 + j;                        // its cache position
     const uint32_t lanes = uint32_t(32 * qd) << 16;
+    const uint32_t tS = tmem + 128 * x + lanes;     // this row's S (and P) in tensor memory
+    const uint32_t tO = tmem + 256 + 128 * x + lanes;
     const float qscale = p.qscale;
     float m_ref = NEG_INF_F, l = 0.f;
     bool ok = true;
     for (int t = 0; t < ntk; ++t) {
-        ok = __all_sync(0xffffffffu, !s_abort && mbar_wait(s_full, t & 1, p.wait_limit_ns));
+        ok = __all_sync(0xffffffffu, !s_abort && mbar_wait(&s_full[x], t & 1, p.wait_limit_ns));
         if (!ok) break;
         tc_fence_after();
+        const int key0 = t * S::TK;
         uint32_t u[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32_nowait(tS + lanes + uint32_t(c * 32), u[c]);
+        for (int c = 0; c < 4; ++c) tmem_ld32_nowait(tS + uint32_t(c * 32), u[c]);
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);
-
-        const int key0 = t * S::TK;
-        float mx = NEG_INF_F;
         if (key0 + S::TK - 1 > qpos_first) {  // tile reaches past some row's position: mask
 #pragma unroll
-            for (int c = 0; c < S::TK; ++c) {
-                float v = __uint_as_float(u[c >> 5][c & 31]);
-                v = (key0 + c <= qpos) ? v : NEG_INF_F;
-                u[c >> 5][c & 31] = __float_as_uint(v);
-                mx = fmaxf(mx, v);
-            }
-        } else {
-#pragma unroll
-            for (int c = 0; c < S::TK; ++c) mx = fmaxf(mx, __uint_as_float(u[c >> 5][c & 31]));
+            for (int c = 0; c < S::TK; ++c)
+                if (key0 + c > qpos) u[c >> 5][c & 31] = __float_as_uint(NEG_INF_F);
         }
+        float mx4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx4[i] = __uint_as_float(u[0][i]);
+#pragma unroll
+        for (int c = 4; c < S::TK; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(u[c >> 5][c & 31]));
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
         const float m_new = fmaxf(m_ref, mx * qscale);
         const bool rescale = m_new > m_ref + S::RESCALE_SLACK;  // also when m_ref = -inf < m_new
         const float corr = rescale ? ex2_approx(m_ref - m_new) : 1.f;
@@ -283,64 +349,73 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             l *= corr;
             m_ref = m_new;
         }
-        const float msub = m_ref == NEG_INF_F ? 0.f : m_ref;
-        uint32_t pw[64];
-        float lsum0 = 0.f, lsum1 = 0.f;
+        // P = 2^(s - m) in bf16 into columns 0..63 of S (keys 2c, 2c + 1 in column c; S is
+        // already in registers); every fourth value from the polynomial, the rest from MUFU
+        const float nmsub = m_ref == NEG_INF_F ? 0.f : -m_ref;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-            const float a = ex2_approx(fmaf(__uint_as_float(u[(2 * e) >> 5][(2 * e) & 31]), qscale, -msub));
-            const float c2 = ex2_approx(fmaf(__uint_as_float(u[(2 * e + 1) >> 5][(2 * e + 1) & 31]), qscale, -msub));
-            lsum0 += a;
-            lsum1 += c2;
-            pw[e] = float2_to_bf16x2(a, c2);
+        for (int c = 0; c < 8; ++c) {
+            uint32_t pw[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int k = 16 * c + 2 * e;
+                const float xa = fmaf(__uint_as_float(u[k >> 5][k & 31]), qscale, nmsub);
+                const float xb = fmaf(__uint_as_float(u[k >> 5][(k & 31) + 1]), qscale, nmsub);
+                const float pa = ex2_approx(xa);
+                const float pb = (e & 1) ? exp2_poly(xb) : ex2_approx(xb);
+                ls[(2 * e) & 3] += pa;
+                ls[(2 * e + 1) & 3] += pb;
+                pw[e] = float2_to_bf16x2(pa, pb);
+            }
+            tmem_st8u(tS + uint32_t(c * 8), pw);
         }
-        l += lsum0 + lsum1;
-        if (t > 0) {
-            // P V of the previous tile has finished: O is final for it and P may be overwritten
-            ok = __all_sync(0xffffffffu, mbar_wait(o_done, (t - 1) & 1, p.wait_limit_ns));
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        if (t > 0 && __any_sync(0xffffffffu, rescale)) {
+            // bring O to the new reference (after P, so that S no longer occupies
+            // registers): P V of the previous tile must have finished
+            ok = __all_sync(0xffffffffu, mbar_wait(&o_done[x], (t - 1) & 1, p.wait_limit_ns));
             if (!ok) break;
             tc_fence_after();
-            if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float o[32];
-                    tmem_ld32(tO + lanes + uint32_t(c * 32), o);
+            for (int c = 0; c < 4; ++c) {
+                float o[32];
+                tmem_ld32(tO + uint32_t(c * 32), o);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] *= corr;
-                    tmem_st32(tO + lanes + uint32_t(c * 32), o);
-                }
+                for (int i = 0; i < 32; ++i) o[i] *= corr;
+                tmem_st32(tO + uint32_t(c * 32), o);
             }
         }
-        uint8_t* prow = Ps + r * 128;
-#pragma unroll
-        for (int cc = 0; cc < 16; ++cc)
-            *reinterpret_cast<uint4*>(prow + (cc >> 3) * S::BOXB + (((cc & 7) ^ (r & 7)) << 4)) =
-                make_uint4(pw[4 * cc], pw[4 * cc + 1], pw[4 * cc + 2], pw[4 * cc + 3]);
-        if (key0 + S::TK > kv_len && key0 + r >= kv_len) {
-            // V rows past the sequence hold whatever the cache holds: zero them so
+        if (x == 0 && key0 + S::TK > kv_len) {
+            // V rows past the sequence hold whatever the cache holds: zero them
+            // (once the tile has landed, before either head's P V reads it) so
             // that the zero probabilities of those keys cannot meet a NaN
-            uint8_t* vrow = base + S::KV_OFF + (t & 1) * 2 * S::TILE_BYTES + S::TILE_BYTES + r * 128;
+            ok = __all_sync(0xffffffffu, mbar_wait(&v_full[t & 1], (t >> 1) & 1, p.wait_limit_ns));
+            if (!ok) break;
+            if (key0 + r >= kv_len) {
+                uint8_t* vrow = base + S::V_OFF + (t & 1) * S::TILE_BYTES + r * 128;
 #pragma unroll
-            for (int bx = 0; bx < 2; ++bx)
+                for (int bx = 0; bx < 2; ++bx)
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc)
-                    *reinterpret_cast<uint4*>(vrow + bx * S::BOXB + cc * 16) = make_uint4(0u, 0u, 0u, 0u);
+                    for (int cc = 0; cc < 8; ++cc)
+                        *reinterpret_cast<uint4*>(vrow + bx * S::BOXB + cc * 16) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(&p_full[x]);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (ntk - 1) & 1, p.wait_limit_ns));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[x], (ntk - 1) & 1, p.wait_limit_ns));
     if (ok) {
         tc_fence_after();
         const float inv = l > 0.f ? 1.f / l : 0.f;
         const bool store = j < nq;
-        uint8_t* orow = p.out + ((int64_t(qrow0) + j) * p.hq + h) * int64_t(S::D * 2);
+        uint8_t* orow = p.out + ((int64_t(qrow0) + j) * p.hq + h0 + x) * int64_t(S::D * 2);
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
             float o[32];
-            tmem_ld32(tO + lanes + uint32_t(c * 32), o);
+            tmem_ld32(tO + uint32_t(c * 32), o);
             if (store) {
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {

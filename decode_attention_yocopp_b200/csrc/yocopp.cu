@@ -240,7 +240,7 @@ int32_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     }
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(unsigned(grid), 1, 1);
-    lc.blockDim = dim3(192, 1, 1);
+    lc.blockDim = dim3(PfShape::THREADS, 1, 1);
     lc.dynamicSmemBytes = PfShape::SMEM;
     lc.stream = st;
     cudaLaunchAttribute attr[1];
@@ -622,7 +622,8 @@ int32_t yocopp_prefill_attn(const void* q, const yocopp_cache* cache, const int3
     if (rows + PfShape::TK >= (int64_t(1) << 31)) return YOCOPP_EINVAL;  // tile row coordinates stay 32-bit
     if (total_q == 0 || max_q == 0) return YOCOPP_OK;
     const int q_tiles = (max_q + PfShape::TQ - 1) / PfShape::TQ;
-    const int64_t grid = int64_t(q_tiles) * cache->batch * num_q_heads;
+    const int heads_per_cta = (num_q_heads / cache->num_kv_heads) % 2 == 0 ? 2 : 1;
+    const int64_t grid = int64_t(q_tiles) * cache->batch * (num_q_heads / heads_per_cta);
     if (grid >= (int64_t(1) << 31)) return YOCOPP_EINVAL;
     alignas(64) CUtensorMap tq, tk, tv;
     if (!encode_q3d(&tq, q, num_q_heads, 128, total_q, PfShape::TQ) ||
@@ -639,6 +640,7 @@ int32_t yocopp_prefill_attn(const void* q, const yocopp_cache* cache, const int3
     p.hkv = cache->num_kv_heads;
     p.capacity = cache->capacity;
     p.q_tiles = q_tiles;
+    p.heads_per_cta = heads_per_cta;
     const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(128.f);
     p.qscale = sc * 1.4426950408889634f;
     p.wait_limit_ns = g_wait_limit_ns;
