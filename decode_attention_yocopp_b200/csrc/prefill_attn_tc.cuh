@@ -11,7 +11,8 @@
 //   out[b,j,h] = sum_u softmax_u(scale q . K'_u) V'_u.
 //
 // Work unit: one CTA per (sequence, 128-row query tile, pair of query heads
-// of one KV head), heaviest query tiles first.  The two heads ("a" and "b")
+// of one KV head); the CTAs of one KV head plane run together, heaviest query
+// tiles first.  The two heads ("a" and "b")
 // share every K/V tile the CTA loads, which halves the K/V traffic per FLOP
 // (a lone head per CTA streams 64 KB of K/V per 8.4 MFLOP, more than L2 can
 // feed every SM at tensor-core speed).  With an odd group size each CTA takes
@@ -107,13 +108,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 
     griddep_wait();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // CTA order: KV head planes one after another (sequence-major), and within a
+    // plane the query tiles heaviest first, so that the CTAs resident at any
+    // time stream the K/V tiles of one or two planes and find them in L2
     const int G = p.hq / p.hkv;
     const int units = G / p.heads_per_cta;                         // CTAs per (sequence, KV head, tile)
-    const int per_tile = p.batch * p.hkv * units;
-    const int jt = p.q_tiles - 1 - int(blockIdx.x) / per_tile;     // heaviest (latest) query tiles first
-    const int rem = int(blockIdx.x) % per_tile;
-    const int b = rem / (p.hkv * units);
-    const int g = (rem / units) % p.hkv;
+    const int per_plane = p.q_tiles * units;
+    const int plane = int(blockIdx.x) / per_plane;                 // b * hkv + g
+    const int rem = int(blockIdx.x) % per_plane;
+    const int jt = p.q_tiles - 1 - rem / units;
+    const int b = plane / p.hkv;
+    const int g = plane % p.hkv;
     const int h0 = g * G + (rem % units) * p.heads_per_cta;
     const bool pair = p.heads_per_cta == 2;
     const int nsm = pair ? 8 : 4;                                  // softmax warps in use
@@ -127,11 +132,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     }
     const int p0 = p.pos ? __ldg(p.pos + b) : 0;
     if (nq < 0) {
-        if (tid == 0 && jt == 0 && rem % (p.hkv * units) == 0) record_status(YOCOPP_EDEVICE_CHECK);
+        if (tid == 0 && jt == 0 && g == 0 && rem % units == 0) record_status(YOCOPP_EDEVICE_CHECK);
         return;
     }
     if (p0 < 0 || int64_t(p0) + nq > p.capacity || nq > p.q_tiles * S::TQ) {
-        if (tid == 0 && jt == 0 && rem % (p.hkv * units) == 0) record_status(YOCOPP_ECAPACITY);
+        if (tid == 0 && jt == 0 && g == 0 && rem % units == 0) record_status(YOCOPP_ECAPACITY);
         return;
     }
     if (jt * S::TQ >= nq) return;
