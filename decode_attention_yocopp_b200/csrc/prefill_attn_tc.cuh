@@ -23,7 +23,8 @@
 //   S_x = Q_x K^T  eight tcgen05.mma (M = 128 queries, N = 128 keys, K = 16
 //                  channels), Q and K K-major from their TMA tiles;
 //   softmax        one thread per query row: masks keys past its position,
-//                  forms P = 2^(s - m) against a reference maximum m that
+//                  forms P = 2^(s - m) (its row sum taken over the bf16 values
+//                  the product uses) against a reference maximum m that
 //                  moves only when the row maximum exceeds it by more than 8
 //                  (then O_x and the row sum are rescaled), so P <= 2^8 and
 //                  rescales are rare; P is written as bf16 into the first 64
@@ -68,8 +69,9 @@ struct PfShape {
     static constexpr int K_OFF = 2 * TILE_BYTES;
     static constexpr int V_OFF = K_OFF + KSLOTS * TILE_BYTES;
     static constexpr int BAR_OFF = V_OFF + VSLOTS * TILE_BYTES;
-    // q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2], o_done[2], drain
-    static constexpr int NBAR = 16;
+    // q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2], o_done[2], drain,
+    // o_last[2]
+    static constexpr int NBAR = 18;
     static constexpr int SMEM = 1024 + BAR_OFF + NBAR * 8 + 16;
     static constexpr int THREADS = 320;
     static constexpr uint32_t IDESC_QK = umma_idesc_bf16(128, 128, false);
@@ -156,6 +158,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     uint64_t* p_full = bars + 11;   // [head]
     uint64_t* o_done = bars + 13;   // [head]
     uint64_t* drain = bars + 15;
+    uint64_t* o_last = bars + 16;   // [head]: the CTA's last P V
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + S::BAR_OFF + S::NBAR * 8);
 
     if (tid == 0) {
@@ -170,6 +173,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             mbar_init(&o_done[s], 1);
         }
         mbar_init(drain, 1);
+        mbar_init(&o_last[0], 1);
+        mbar_init(&o_last[1], 1);
         fence_mbar_init();
         s_abort = 0;
         s_cdone = 0;
@@ -257,6 +262,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                                      umma_desc_sw128_mn(va + uint32_t(kk * 16 * 128), S::BOXB, 1024), S::IDESC_PV,
                                      (t > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(&o_done[x]);
+                if (t == ntk - 1) umma_commit(&o_last[x]);
                 issued_any = true;
             };
             if (ok) ok = !s_abort && mbar_wait(&k_full[0], 0, p.wait_limit_ns);
@@ -355,9 +361,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             m_ref = m_new;
         }
         // P = 2^(s - m) in bf16 into columns 0..63 of S (keys 2c, 2c + 1 in column c; S is
-        // already in registers); every fourth value from the polynomial, the rest from MUFU
+        // already in registers); every fourth value from the polynomial, the rest from MUFU.
+        // The row sum adds the bf16 values the product uses, so that the output is a convex
+        // combination of V rows: its error is then sum_u w_u e_u (V_u - out) (e_u the relative
+        // rounding of P_u), which vanishes where one key dominates.
         const float nmsub = m_ref == NEG_INF_F ? 0.f : -m_ref;
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             uint32_t pw[8];
@@ -368,13 +377,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 const float xb = fmaf(__uint_as_float(u[k >> 5][(k & 31) + 1]), qscale, nmsub);
                 const float pa = ex2_approx(xa);
                 const float pb = (e & 1) ? exp2_poly(xb) : ex2_approx(xb);
-                ls[(2 * e) & 3] += pa;
-                ls[(2 * e + 1) & 3] += pb;
                 pw[e] = float2_to_bf16x2(pa, pb);
+                ls[e & 1] = fadd2(ls[e & 1], bf16x2_to_float2(pw[e]));
             }
             tmem_st8u(tS + uint32_t(c * 8), pw);
         }
-        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        l += (ls[0].x + ls[1].x) + (ls[0].y + ls[1].y);
         if (t > 0 && __any_sync(0xffffffffu, rescale)) {
             // bring O to the new reference (after P, so that S no longer occupies
             // registers): P V of the previous tile must have finished
@@ -411,7 +419,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[x]);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[x], (ntk - 1) & 1, p.wait_limit_ns));
+    // O is final once the CTA's last P V for this head has completed (a one-phase barrier,
+    // so the wait cannot be confused by phase parity)
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_last[x], 0, p.wait_limit_ns));
     if (ok) {
         tc_fence_after();
         const float inv = l > 0.f ? 1.f / l : 0.f;
