@@ -366,21 +366,22 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         // combination of V rows: its error is then sum_u w_u e_u (V_u - out) (e_u the relative
         // rounding of P_u), which vanishes where one key dominates.
         const float nmsub = m_ref == NEG_INF_F ? 0.f : -m_ref;
+        const float2 qs2 = make_float2(qscale, qscale), nm2 = make_float2(nmsub, nmsub);
         float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            uint32_t pw[8];
+        for (int c = 0; c < 2; ++c) {
+            uint32_t pw[32];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int k = 16 * c + 2 * e;
-                const float xa = fmaf(__uint_as_float(u[k >> 5][k & 31]), qscale, nmsub);
-                const float xb = fmaf(__uint_as_float(u[k >> 5][(k & 31) + 1]), qscale, nmsub);
-                const float pa = ex2_approx(xa);
-                const float pb = (e & 1) ? exp2_poly(xb) : ex2_approx(xb);
+            for (int e = 0; e < 32; ++e) {
+                const int k = 64 * c + 2 * e;
+                const float2 xv = ffma2(make_float2(__uint_as_float(u[k >> 5][k & 31]),
+                                                    __uint_as_float(u[k >> 5][(k & 31) + 1])), qs2, nm2);
+                const float pa = ex2_approx(xv.x);
+                const float pb = (e & 1) ? exp2_poly(xv.y) : ex2_approx(xv.y);
                 pw[e] = float2_to_bf16x2(pa, pb);
                 ls[e & 1] = fadd2(ls[e & 1], bf16x2_to_float2(pw[e]));
             }
-            tmem_st8u(tS + uint32_t(c * 8), pw);
+            tmem_st32u(tS + uint32_t(c * 32), pw);
         }
         l += (ls[0].x + ls[1].x) + (ls[0].y + ls[1].y);
         if (t > 0 && __any_sync(0xffffffffu, rescale)) {
