@@ -437,7 +437,7 @@ def run_ours(args, rank, world, local):
     del step.raw_shared, step.fused_ws
 
     prefill = None
-    if not args.no_prefill and w.dtype == "bf16" and w.d == 128 and not w.paged:
+    if not args.no_prefill and w.dtype == "bf16" and w.d == 128:
         prefill = run_prefill_attention(args, step, world)
 
     e2e = None

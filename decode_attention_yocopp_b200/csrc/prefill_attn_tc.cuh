@@ -52,8 +52,11 @@ struct PrefillParams {
     uint8_t* out;           // [total_q][hq][128] bf16
     const int32_t* pos;     // [batch] cache position of each sequence's first query row, or null (0)
     const int32_t* cu_q;    // [batch + 1] query-row offsets, or null (n_uniform rows per sequence)
+    const int32_t* block_table;  // [batch][mbps] for a paged cache, or null (contiguous)
     int32_t n_uniform;
     int32_t batch, hq, hkv, capacity;
+    int32_t block_size, mbps, num_blocks;  // paged cache only
+    int32_t boxr;           // rows per K/V box: 128 (contiguous) or min(block_size, 128)
     int32_t q_tiles;        // ceil(max query rows per sequence / 128)
     int32_t heads_per_cta;  // 2 (group size even) or 1
     float qscale;           // softmax scale * log2(e)
@@ -208,16 +211,40 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                                     h0 + x, qrow0 + jt * S::TQ);
             }
             const int plane_row = (b * p.hkv + g) * p.capacity;
+            const int nsb = S::TK / p.boxr;  // boxes of boxr rows per tile (one per cache block)
             for (int t = 0; t < ntk; ++t) {
                 const int slot = t & 1;
                 if (s_abort || !mbar_wait(&empty[slot], ((t >> 1) & 1) ^ 1, p.wait_limit_ns)) {
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(&full[slot], uint32_t(S::TILE_BYTES));
-                for (int bx = 0; bx < 2; ++bx)
-                    tma_load_2d(ring + slot * S::TILE_BYTES + bx * S::BOXB, map, &full[slot], bx * 64,
-                                plane_row + t * S::TK);
+                // the tile's rows: one 128-row box (contiguous), or one box per cache block;
+                // blocks wholly past the sequence are not loaded (their K rows are masked and
+                // their V rows zeroed before use)
+                int rows[S::TK / 16];
+                int nb = 0;
+                for (int sb = 0; sb < nsb; ++sb) {
+                    const int tok = t * S::TK + sb * p.boxr;
+                    int row = -1;
+                    if (p.block_table == nullptr) {
+                        row = plane_row + tok;
+                    } else if (tok < kv_len) {
+                        const int blk = __ldg(p.block_table + int64_t(b) * p.mbps + tok / p.block_size);
+                        if (blk < 0 || blk >= p.num_blocks)
+                            record_status(YOCOPP_EDEVICE_CHECK);
+                        else
+                            row = (blk * p.hkv + g) * p.block_size + tok % p.block_size;
+                    }
+                    rows[sb] = row;
+                    nb += row >= 0;
+                }
+                mbar_arrive_expect_tx(&full[slot], uint32_t(nb * p.boxr * 2 * 128));
+                for (int sb = 0; sb < nsb; ++sb) {
+                    if (rows[sb] < 0) continue;
+                    for (int bx = 0; bx < 2; ++bx)
+                        tma_load_2d(ring + slot * S::TILE_BYTES + bx * S::BOXB + sb * p.boxr * 128, map, &full[slot],
+                                    bx * 64, rows[sb]);
+                }
                 issued = t + 1;
             }
             if (!ok) {

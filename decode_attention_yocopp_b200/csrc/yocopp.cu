@@ -606,7 +606,8 @@ int32_t yocopp_prefill_attn(const void* q, const yocopp_cache* cache, const int3
     const int32_t rc = check_cache(cache);
     if (rc != YOCOPP_OK) return rc;
     if (cache->dtype != YOCOPP_BF16) return YOCOPP_EDTYPE;
-    if (cache->head_dim != 128 || cache->block_table != nullptr) return YOCOPP_EINVAL;
+    if (cache->head_dim != 128) return YOCOPP_EINVAL;
+    const bool paged = cache->block_table != nullptr;
     if (num_q_heads < 1 || num_q_heads % cache->num_kv_heads != 0) return YOCOPP_EINVAL;
     if (q == nullptr || out == nullptr || !aligned(q, 16) || !aligned(out, 16)) return YOCOPP_EINVAL;
     if (!(scale >= 0.f) || !std::isfinite(scale)) return YOCOPP_EINVAL;
@@ -618,8 +619,10 @@ int32_t yocopp_prefill_attn(const void* q, const yocopp_cache* cache, const int3
         return YOCOPP_EINVAL;
     }
     if (int64_t(max_q) > int64_t(cache->capacity)) return YOCOPP_EINVAL;
-    const int64_t rows = int64_t(cache->batch) * cache->num_kv_heads * cache->capacity;
+    const int64_t rows = paged ? int64_t(cache->num_blocks) * cache->num_kv_heads * cache->block_size
+                               : int64_t(cache->batch) * cache->num_kv_heads * cache->capacity;
     if (rows + PfShape::TK >= (int64_t(1) << 31)) return YOCOPP_EINVAL;  // tile row coordinates stay 32-bit
+    const int boxr = paged ? (cache->block_size < PfShape::TK ? cache->block_size : PfShape::TK) : PfShape::TK;
     if (total_q == 0 || max_q == 0) return YOCOPP_OK;
     const int q_tiles = (max_q + PfShape::TQ - 1) / PfShape::TQ;
     const int heads_per_cta = (num_q_heads / cache->num_kv_heads) % 2 == 0 ? 2 : 1;
@@ -627,13 +630,18 @@ int32_t yocopp_prefill_attn(const void* q, const yocopp_cache* cache, const int3
     if (grid >= (int64_t(1) << 31)) return YOCOPP_EINVAL;
     alignas(64) CUtensorMap tq, tk, tv;
     if (!encode_q3d(&tq, q, num_q_heads, 128, total_q, PfShape::TQ) ||
-        !encode_rows(&tk, cache->k, YOCOPP_BF16, 128, rows, PfShape::TK) ||
-        !encode_rows(&tv, cache->v, YOCOPP_BF16, 128, rows, PfShape::TK))
+        !encode_rows(&tk, cache->k, YOCOPP_BF16, 128, rows, boxr) ||
+        !encode_rows(&tv, cache->v, YOCOPP_BF16, 128, rows, boxr))
         return YOCOPP_ECUDA;
     PrefillParams p;
     p.out = static_cast<uint8_t*>(out);
     p.pos = pos;
     p.cu_q = cu_q;
+    p.block_table = cache->block_table;
+    p.block_size = paged ? cache->block_size : 0;
+    p.mbps = paged ? cache->max_blocks_per_seq : 0;
+    p.num_blocks = paged ? cache->num_blocks : 0;
+    p.boxr = boxr;
     p.n_uniform = cu_q ? 0 : n_uniform;
     p.batch = cache->batch;
     p.hq = num_q_heads;

@@ -86,7 +86,7 @@ class SharedKVStack:
                        cu_q: Optional[torch.Tensor] = None, n_uniform: int = 0, max_q: int = 0,
                        scale: float = 0.0, stream=None) -> torch.Tensor:
         """Self-decoder layer i's causal prefill attention over its own cache, after
-        ``write`` has appended the same tokens (bf16, head_dim 128, contiguous)."""
+        ``write`` has appended the same tokens (bf16, head_dim 128, contiguous or paged)."""
         yocopp_prefill_attn(q, self.desc[i], out, pos=pos, cu_q=cu_q, n_uniform=n_uniform, total_q=q.shape[0],
                             max_q=max_q, num_q_heads=self.hq, scale=scale, stream=stream)
         return out

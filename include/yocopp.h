@@ -263,9 +263,11 @@ int32_t yocopp_decode_attn_static(const void* q, const yocopp_cache* cache, cons
  *             token-major and packed over the batch like yocopp_compose_append's
  *             inputs: sequence b's rows are [cu_q[b], cu_q[b+1]) or, when
  *             cu_q == NULL, [b * n_uniform, (b + 1) * n_uniform).
- *   cache   : HOST descriptor; bf16, head_dim 128, contiguous (block_table
- *             NULL).  Positions [0, p_b + n_b) of sequence b must hold the
- *             composed rows.
+ *   cache   : HOST descriptor; bf16, head_dim 128, contiguous or paged (any
+ *             block size yocopp_cache allows).  Positions [0, p_b + n_b) of
+ *             sequence b must hold the composed rows; a block-table entry
+ *             outside [0, num_blocks) for such a position records
+ *             YOCOPP_EDEVICE_CHECK (that block is not read).
  *   pos     : device int32 [batch] or NULL (all 0; a whole-prompt prefill).
  *   cu_q    : device int32 [batch + 1] prefix offsets, or NULL.
  *   n_uniform : rows per sequence when cu_q == NULL.

@@ -94,7 +94,7 @@ def test_prefill_host_checks():
                                    None) == y.YOCOPP_EDTYPE
     assert lib.yocopp_prefill_attn(0x10, ctypes.byref(_cache(head_dim=64)), None, None, 4, 8, 0, 0x10, 32, 0.0,
                                    None) == y.YOCOPP_EINVAL
-    paged = _cache(block_table=0x3000, block_size=64, max_blocks_per_seq=1, num_blocks=4)
+    paged = _cache(block_table=0x3000, block_size=48, max_blocks_per_seq=1, num_blocks=4, capacity=48)
     assert lib.yocopp_prefill_attn(0x10, ctypes.byref(paged), None, None, 4, 8, 0, 0x10, 32, 0.0, None) == y.YOCOPP_EINVAL
     # query heads, pointers, alignment, scale, counts
     assert lib.yocopp_prefill_attn(0x10, ctypes.byref(c), None, None, 4, 8, 0, 0x10, 12, 0.0, None) == y.YOCOPP_EINVAL

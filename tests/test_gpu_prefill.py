@@ -17,7 +17,7 @@ import torch
 
 import gen
 import oracle
-from gpu_util import assert_attention, fill_sentinel, np_storage, scatter_rows, to_device
+from gpu_util import assert_attention, fill_sentinel, np_storage, random_block_table, scatter_rows, to_device
 from oracle import model
 
 pytestmark = pytest.mark.gpu
@@ -43,15 +43,24 @@ def _bf16_rows(rng, shape, scale=1.0):
 
 
 def run_case(y, orc, *, hkv, G, nq, pos=None, capacity=None, uniform=None, key_scale=1.5, seed=1,
-             scale=0.0, pass_pos=True):
-    """Prefill rows nq[b] of each sequence at cache positions pos[b]..; compare all outputs."""
+             scale=0.0, pass_pos=True, block_size=None):
+    """Prefill rows nq[b] of each sequence at cache positions pos[b]..; compare all outputs.
+    block_size selects a paged cache (random block table over a pool with spare blocks)."""
     rng = np.random.default_rng(seed)
     B = len(nq)
     hq = hkv * G
     p0 = list(pos) if pos is not None else [0] * B
     kv_len = [a + n for a, n in zip(p0, nq)]
     cap = capacity or max(1, max(kv_len))
-    kc = torch.empty((B, hkv, cap, D), dtype=torch.bfloat16, device="cuda")
+    bt = None
+    if block_size:
+        mbps = (cap + block_size - 1) // block_size
+        cap = mbps * block_size
+        nblocks = B * mbps + 3
+        bt = random_block_table(rng, B, mbps, nblocks)
+        kc = torch.empty((nblocks, hkv, block_size, D), dtype=torch.bfloat16, device="cuda")
+    else:
+        kc = torch.empty((B, hkv, cap, D), dtype=torch.bfloat16, device="cuda")
     vc = torch.empty_like(kc)
     fill_sentinel(kc)
     fill_sentinel(vc)
@@ -61,15 +70,15 @@ def run_case(y, orc, *, hkv, G, nq, pos=None, capacity=None, uniform=None, key_s
         for g in range(hkv):
             K[b, g] = _bf16_rows(rng, (kv_len[b], D), key_scale)
             V[b, g] = _bf16_rows(rng, (kv_len[b], D))
-            scatter_rows(kc, K[b, g], b, g, None, "bf16")
-            scatter_rows(vc, V[b, g], b, g, None, "bf16")
+            scatter_rows(kc, K[b, g], b, g, bt, "bf16")
+            scatter_rows(vc, V[b, g], b, g, bt, "bf16")
     cu = np.concatenate([[0], np.cumsum(nq)]).astype(np.int64)
     total = int(cu[-1])
     qbits = _bf16_rows(rng, (max(1, total), hq, D))[:total]
     q = to_device(qbits, "bf16") if total else torch.empty((0, hq, D), dtype=torch.bfloat16, device="cuda")
     out = torch.empty((total, hq, D), dtype=torch.bfloat16, device="cuda")
     fill_sentinel(out)
-    cache = y.make_cache(kc, vc)
+    cache = y.make_cache(kc, vc, torch.from_numpy(bt).cuda() if bt is not None else None)
     is_uniform = len(set(nq)) == 1 if uniform is None else uniform
     pos_t = torch.tensor(p0, dtype=torch.int32, device="cuda") if pass_pos else None
     if is_uniform:
@@ -125,6 +134,32 @@ def test_peaked_logits_and_explicit_scale(y, orc):
 
 def test_group_of_eight(y, orc):
     run_case(y, orc, hkv=1, G=8, nq=[150], seed=6)
+
+
+@pytest.mark.parametrize("bs", [16, 64, 128, 256])
+def test_paged_cache(y, orc, bs):
+    # a shuffled block table; ragged rows with offsets, tiles that span several blocks,
+    # sequences that end inside a block (the rest of the pool stays NaN)
+    run_case(y, orc, hkv=2, G=4, nq=[300, 1, 129, 200], pos=[0, 40, 70, 3], block_size=bs, seed=20 + bs)
+
+
+def test_paged_single_head_mode(y, orc):
+    run_case(y, orc, hkv=2, G=1, nq=[257, 64], pos=[0, 100], block_size=64, seed=31)
+
+
+def test_invalid_block_is_reported(y, orc):
+    """A block-table entry outside the pool for a position in use records
+    YOCOPP_EDEVICE_CHECK (the block is not read)."""
+    rng = np.random.default_rng(9)
+    hkv, bs = 1, 64
+    kc = torch.from_numpy(_bf16_rows(rng, (4, hkv, bs, D)).view(np.int16)).cuda().view(torch.bfloat16)
+    vc = torch.from_numpy(_bf16_rows(rng, (4, hkv, bs, D)).view(np.int16)).cuda().view(torch.bfloat16)
+    bt = torch.tensor([[0, 9]], dtype=torch.int32, device="cuda")  # block 9 is outside the 4-block pool
+    q = to_device(_bf16_rows(rng, (100, 2, D)), "bf16")
+    out = torch.empty((100, 2, D), dtype=torch.bfloat16, device="cuda")
+    y.yocopp_get_device_status(reset=True)
+    y.yocopp_prefill_attn(q, y.make_cache(kc, vc, bt), out, n_uniform=100, total_q=100)
+    assert y.yocopp_get_device_status(reset=True) == y.YOCOPP_EDEVICE_CHECK
 
 
 def test_out_of_capacity_is_reported(y, orc):
@@ -212,26 +247,45 @@ def test_e2e_b32_t8192_sampled(y, orc):
     _e2e_sampled_sequences(y, orc, w, w.shared_layer, seqs=[0, 17, 31], rows_per_seq=6)
 
 
+def test_e2e_ragged64_paged_sampled(y, orc):
+    # the ragged serving batch: 64 lengths in [512, 32768], paged cache (block 64, shuffled pool)
+    w = gen.config(5)
+    _e2e_sampled_sequences(y, orc, w, w.shared_layer, seqs=[0, int(np.argmax(w.lens)), 63], rows_per_seq=4)
+
+
 def _e2e_sampled_sequences(y, orc, w, layer, seqs, rows_per_seq):
     """As _e2e at full size, checking only a few sequences (the oracle's cost)."""
     from decode_attention_yocopp_b200.pipeline import SharedKVStack
-    stack = SharedKVStack(w.layers, w.batch, w.hq, w.hkv, w.d, torch.bfloat16, w.alpha, w.lam,
-                          capacity=max(1, w.max_len), cache_layers=[layer])
+    if w.paged:
+        bt = torch.from_numpy(w.block_table()).cuda()
+        stack = SharedKVStack(w.layers, w.batch, w.hq, w.hkv, w.d, torch.bfloat16, w.alpha, w.lam, block_table=bt,
+                              block_size=w.block_size, num_blocks=w.num_blocks, cache_layers=[layer])
+    else:
+        stack = SharedKVStack(w.layers, w.batch, w.hq, w.hkv, w.d, torch.bfloat16, w.alpha, w.lam,
+                              capacity=max(1, w.max_len), cache_layers=[layer])
     pos0 = torch.zeros(w.batch, dtype=torch.int32, device="cuda")
+    cu = torch.from_numpy(w.cu_prefill.astype(np.int32)).cuda()
     k1, v1 = w.device(gen.K_PREFILL, 1), w.device(gen.V_PREFILL, 1)
-    stack.write(layer, k1, v1, w.device(gen.K_PREFILL, layer), w.device(gen.V_PREFILL, layer), pos0,
-                n_uniform=w.prefill_lens[0])
-    del k1, v1
+    ki, vi = w.device(gen.K_PREFILL, layer), w.device(gen.V_PREFILL, layer)
+    if w.uniform:
+        stack.write(layer, k1, v1, ki, vi, pos0, n_uniform=w.prefill_lens[0])
+    else:
+        stack.write(layer, k1, v1, ki, vi, pos0, cu_new=cu)
+    del k1, v1, ki, vi
     q = w.device(gen.Q_PREFILL, layer)
     out = torch.empty_like(q)
     fill_sentinel(out)
-    stack.prefill_attend(layer, q, out, n_uniform=w.prefill_lens[0])
+    if w.uniform:
+        stack.prefill_attend(layer, q, out, n_uniform=w.prefill_lens[0])
+    else:
+        stack.prefill_attend(layer, q, out, cu_q=cu, max_q=max(w.prefill_lens))
     torch.cuda.synchronize()
     assert y.yocopp_get_device_status(reset=True) == 0
     rng = np.random.default_rng(2)
-    n = w.prefill_lens[0]
     for b in seqs:
+        n = w.prefill_lens[b]
         rows = np.unique(np.concatenate([[0, 128, n - 1], rng.integers(0, n, rows_per_seq)]))
+        rows = rows[rows < n]
         got_b = np_storage(out[int(w.cu_prefill[b]) + torch.from_numpy(rows).cuda()])
         for g in (0, w.hkv - 1):
             kv = (model.composed_seq(orc, w, layer, "K", b, g)[:n], model.composed_seq(orc, w, layer, "V", b, g)[:n])
