@@ -87,3 +87,23 @@ def test_peak_fallback(tmp_path, monkeypatch):
     assert bench.hbm_peak() == (bench.FALLBACK_HBM_GBS, "fallback")
     (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6441.9}))
     assert bench.hbm_peak() == (6441.9, "measured")
+
+
+def test_causal_pair_count():
+    # whole-prompt causal prefill: a sequence of n rows scores n (n + 1) / 2 (query, key) pairs
+    assert bench.causal_pairs([]) == 0
+    assert bench.causal_pairs([1]) == 1
+    assert bench.causal_pairs([3, 1, 0]) == 6 + 1
+    n = 8191
+    assert bench.causal_pairs([n] * 32) == 32 * n * (n + 1) // 2
+    # brute-force count of u <= t for a small case
+    assert bench.causal_pairs([7, 5]) == sum(1 for n in (7, 5) for t in range(n) for u in range(n) if u <= t)
+
+
+def test_tensor_peak_reads_measured_file(tmp_path, monkeypatch):
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"bf16_tflops": 1000.0, "bf16_tflops_sustained": 900.0}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.tensor_peak() == (1000.0, 900.0, "measured")
+    (tmp_path / "MEASURED_PEAKS.json").unlink()
+    burst, sustained, kind = bench.tensor_peak()
+    assert kind == "fallback" and burst > sustained > 0
