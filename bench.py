@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode-attn KV-read GB/s (% of B200 HBM peak); compose GB/s; decode tok/s"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (reported beside the measured copy peak)
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -463,12 +464,14 @@ def run_ours(args, rank, world, local):
     workload = f"{w.name}"
     roof_comp = {"kernel": "compose_append_kernel (prefill size)", "bound": "hbm", "achieved": round(ach_comp, 1),
                  "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(ach_comp / peak, 4),
+                 "frac_of_nominal": round(ach_comp / NOMINAL_HBM_GBS, 4),
                  "traffic": ncu_traffic("compose_append_kernel", workload),
                  "algorithmic_bytes_per_launch": w.compose_bytes(w.total_prefill)}
     dk = decode_kernel_name(w, args.decode_kernel)
     roof_attn = {"kernel": f"{dk} (one layer, split + merge)", "bound": "hbm",
                  "achieved": round(ach_attn, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                 "frac": round(ach_attn / peak, 4), "traffic": ncu_traffic(dk, workload),
+                 "frac": round(ach_attn / peak, 4), "frac_of_nominal": round(ach_attn / NOMINAL_HBM_GBS, 4),
+                 "traffic": ncu_traffic(dk, workload),
                  "algorithmic_bytes_per_launch": kv_bytes_layer}
     dominant = roof_comp if t_prefill >= t_attn else roof_attn
     line = {
@@ -676,10 +679,14 @@ def oracle_sample(w, seconds: float, threads: int):
 def cpu_baseline(w, seconds):
     threads = _cpu_threads()
     kv, comp, el, n = oracle_sample(w, seconds, threads)
+    # the same work on one core, on a shorter sample
+    kv1, _, el1, n1 = oracle_sample(w, max(2.0, seconds / 4), 1)
     return {"value": round(kv / el / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"{n} (sequence, kv-head) planes of {w.name}: fp64 compose of the shared layer's plane "
                       f"+ one cross-decoder layer's attention over it, {el:.1f} s",
-            "compose_gbs": round(comp / el / 1e9, 4)}
+            "compose_gbs": round(comp / el / 1e9, 4),
+            "single_core": {"value": round(kv1 / el1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                            "sample": f"{n1} planes, {el1:.1f} s"}}
 
 
 def run_reference(args, rank, world):
