@@ -61,6 +61,7 @@ struct PrefillParams {
     int32_t heads_per_cta;  // 2 (group size even) or 1
     float qscale;           // softmax scale * log2(e)
     uint64_t wait_limit_ns;
+    int32_t drop_k_tile;    // testing: K tile whose load CTA 0 never issues (-1: none)
 };
 
 struct PfShape {
@@ -218,6 +219,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     ok = false;
                     break;
                 }
+                if (kl && t == p.drop_k_tile && blockIdx.x == 0) continue;  // failure injection (tests)
                 // the tile's rows: one 128-row box (contiguous), or one box per cache block;
                 // blocks wholly past the sequence are not loaded (their K rows are masked and
                 // their V rows zeroed before use)

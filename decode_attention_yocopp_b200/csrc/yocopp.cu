@@ -652,6 +652,7 @@ int32_t yocopp_prefill_attn(const void* q, const yocopp_cache* cache, const int3
     const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(128.f);
     p.qscale = sc * 1.4426950408889634f;
     p.wait_limit_ns = g_wait_limit_ns;
+    p.drop_k_tile = g_test_drop_tile;
     return launch_prefill(tq, tk, tv, p, grid, static_cast<cudaStream_t>(stream));
 }
 

@@ -314,12 +314,15 @@ int32_t yocopp_set_decode_kernel(int32_t which);
 
 /*
  * yocopp_testing_set_decode_fault - failure-injection hook for tests.
- * Host-side, process-wide; affects later yocopp_decode_attn launches.
- *   drop_tile     : index (in the split plan's flattened tile order) of one
- *                   tile whose load is never issued, so the consumers' wait on
- *                   it can only run out; -1 disables the injection.
- *   wait_limit_ns : limit of every bounded wait inside the decode kernel
- *                   (default 2 s); must be > 0.
+ * Host-side, process-wide; affects later yocopp_decode_attn and
+ * yocopp_prefill_attn launches.
+ *   drop_tile     : decode: index (in the split plan's flattened tile order) of
+ *                   one tile whose load is never issued, so the consumers' wait
+ *                   on it can only run out; prefill: index of the key tile
+ *                   whose K load the first CTA never issues; -1 disables the
+ *                   injection.
+ *   wait_limit_ns : limit of every bounded wait inside the decode and prefill
+ *                   kernels (default 2 s); must be > 0.
  * With a dropped tile the kernel records YOCOPP_ETIMEOUT, waits (bounded) for
  * its own copies still in flight, and returns; the context stays usable.
  * Returns YOCOPP_EINVAL for wait_limit_ns <= 0.

@@ -162,6 +162,26 @@ def test_invalid_block_is_reported(y, orc):
     assert y.yocopp_get_device_status(reset=True) == y.YOCOPP_EDEVICE_CHECK
 
 
+def test_dropped_tile_times_out_and_recovers(y, orc):
+    """A K tile whose load is never issued (failure injection) makes the first CTA's
+    bounded waits run out: the call records YOCOPP_ETIMEOUT, the kernel ends, and the
+    next call (injection off) is correct."""
+    try:
+        y.yocopp_testing_set_decode_fault(1, 50_000_000)  # drop key tile 1 of CTA 0; 50 ms waits
+        rng = np.random.default_rng(12)
+        n = 300
+        kc = torch.from_numpy(_bf16_rows(rng, (1, 2, n, D)).view(np.int16)).cuda().view(torch.bfloat16)
+        vc = torch.from_numpy(_bf16_rows(rng, (1, 2, n, D)).view(np.int16)).cuda().view(torch.bfloat16)
+        q = to_device(_bf16_rows(rng, (n, 4, D)), "bf16")
+        out = torch.empty((n, 4, D), dtype=torch.bfloat16, device="cuda")
+        y.yocopp_get_device_status(reset=True)
+        y.yocopp_prefill_attn(q, y.make_cache(kc, vc), out, n_uniform=n, total_q=n)
+        assert y.yocopp_get_device_status(reset=True) == y.YOCOPP_ETIMEOUT
+    finally:
+        y.yocopp_testing_set_decode_fault(-1, 2_000_000_000)
+    run_case(y, orc, hkv=2, G=2, nq=[300], seed=13)
+
+
 def test_out_of_capacity_is_reported(y, orc):
     """A sequence whose rows would pass the cache capacity is skipped (its output
     rows keep their contents) and YOCOPP_ECAPACITY is recorded; others run."""
