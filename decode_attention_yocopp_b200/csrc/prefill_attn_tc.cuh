@@ -85,24 +85,50 @@ struct PfShape {
 };
 static_assert(PfShape::SMEM <= 232448 - 16, "prefill shared memory");
 
-// 2^x on the FMA pipe, for x <= 2^22 (x below -126 is taken as -126, whose
-// result, at most 2^-125.5, is nothing next to the row's largest term 1):
-// x = j + f with j = round(x), f in [-1/2, 1/2] (Cody and Waite's range
-// reduction, with the round done by adding 1.5 * 2^23), 2^f from a cubic
-// fitted here to the relative error on [-1/2, 1/2] (max 7.5e-5, far below
-// the 2^-9 of the bf16 probabilities it feeds), and 2^j added to the exponent
-// field.  The exponential unit does 16 results per clock per SM, one tile's
-// worth in the time the tensor cores take for it; moving a quarter of them
-// here keeps it off the critical path.
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -126.f);  // keeps the exponent field of the result >= 0
-    const float t = x + 12582912.f;          // 1.5 * 2^23: round to integer in the low mantissa bits
-    const float f = x - (t - 12582912.f);
-    float p = fmaf(0x1.c3f76p-5f, f, 0x1.f0de1ap-3f);
-    p = fmaf(p, f, 0x1.62f31ap-1f);
-    p = fmaf(p, f, 0x1.fff692p-1f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+// 2^x on the FMA pipe for two arguments at once (fp32x2 arithmetic), for
+// x <= 2^22 (x below -126 is taken as -126, whose result, at most 2^-125.5,
+// is nothing next to the row's largest term 1): x = j + f with j = round(x),
+// f in [-1/2, 1/2] (Cody and Waite's range reduction, with the round done by
+// adding 1.5 * 2^23), 2^f from a cubic fitted here to the relative error on
+// [-1/2, 1/2] (max 7.5e-5, far below the 2^-9 of the bf16 probabilities it
+// feeds), and 2^j added to the exponent field.  The exponential unit does 16
+// results per clock per SM, one tile's worth in the time the tensor cores take
+// for it; moving a quarter of them here keeps it off the critical path.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    x.x = fmaxf(x.x, -126.f);  // keeps the exponent field of the result >= 0
+    x.y = fmaxf(x.y, -126.f);
+    const float2 mg = make_float2(12582912.f, 12582912.f), nmg = make_float2(-12582912.f, -12582912.f);
+    const float2 t = fadd2(x, mg);                                      // round(x) in the low mantissa bits
+    const float2 f = ffma2(fadd2(t, nmg), make_float2(-1.f, -1.f), x);  // x - round(x), exact
+    float2 p = ffma2(make_float2(0x1.c3f76p-5f, 0x1.c3f76p-5f), f, make_float2(0x1.f0de1ap-3f, 0x1.f0de1ap-3f));
+    p = ffma2(p, f, make_float2(0x1.62f31ap-1f, 0x1.62f31ap-1f));
+    p = ffma2(p, f, make_float2(0x1.fff692p-1f, 0x1.fff692p-1f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
+
+// max of three (sm_100 three-input max.f32; a NaN input is skipped as by fmaxf)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// acc + the two bf16 of w (low half into .x), each widened exactly and added
+// with one rounding (sm_100 mixed-precision add.f32.bf16): the sums that
+// widening first and adding in fp32 give, without the widening instructions.
+__device__ __forceinline__ float2 add_bf16x2(float2 acc, uint32_t w) {
+    float2 r;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %3;\n\tadd.rn.f32.bf16 %1, hi, %4;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "r"(w), "f"(acc.x), "f"(acc.y));
+    return r;
+}
+
+// Pairs of keys whose two exponentials come from the cubic (one pair in four:
+// a quarter of the exponentials on the FMA pipe, the rest on MUFU).
+__device__ __forceinline__ constexpr bool poly_pair(int e) { return (e & 3) == 3; }
 
 __global__ void __launch_bounds__(PfShape::THREADS, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -380,8 +406,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 #pragma unroll
         for (int i = 0; i < 4; ++i) mx4[i] = __uint_as_float(u[0][i]);
 #pragma unroll
-        for (int c = 4; c < S::TK; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(u[c >> 5][c & 31]));
-        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        for (int c = 4; c < S::TK; c += 2)
+            mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(u[c >> 5][c & 31]),
+                                      __uint_as_float(u[c >> 5][(c & 31) + 1]));
+        const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
         const float m_new = fmaxf(m_ref, mx * qscale);
         const bool rescale = m_new > m_ref + S::RESCALE_SLACK;  // also when m_ref = -inf < m_new
         const float corr = rescale ? ex2_approx(m_ref - m_new) : 1.f;
@@ -390,7 +418,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             m_ref = m_new;
         }
         // P = 2^(s - m) in bf16 into columns 0..63 of S (keys 2c, 2c + 1 in column c; S is
-        // already in registers); every fourth value from the polynomial, the rest from MUFU.
+        // already in registers); one pair of keys in four from the polynomial, the rest from MUFU.
         // The row sum adds the bf16 values the product uses, so that the output is a convex
         // combination of V rows: its error is then sum_u w_u e_u (V_u - out) (e_u the relative
         // rounding of P_u), which vanishes where one key dominates.
@@ -405,10 +433,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 const int k = 64 * c + 2 * e;
                 const float2 xv = ffma2(make_float2(__uint_as_float(u[k >> 5][k & 31]),
                                                     __uint_as_float(u[k >> 5][(k & 31) + 1])), qs2, nm2);
-                const float pa = ex2_approx(xv.x);
-                const float pb = (e & 1) ? exp2_poly(xv.y) : ex2_approx(xv.y);
-                pw[e] = float2_to_bf16x2(pa, pb);
-                ls[e & 1] = fadd2(ls[e & 1], bf16x2_to_float2(pw[e]));
+                const float2 pe = poly_pair(e) ? exp2_poly2(xv) : make_float2(ex2_approx(xv.x), ex2_approx(xv.y));
+                pw[e] = float2_to_bf16x2(pe.x, pe.y);
+                ls[e & 1] = add_bf16x2(ls[e & 1], pw[e]);
             }
             tmem_st32u(tS + uint32_t(c * 32), pw);
         }
