@@ -103,7 +103,7 @@ typedef struct yocopp_cache {
  *                    [b * n_uniform, (b + 1) * n_uniform).  K1/V1 are the
  *                    current tokens' layer-1 values (they may alias Ki/Vi).
  *   alpha          : HOST, 4 floats {aK1, aK2, aV1, aV2}.
- *   lambda         : the scale factor (35 in the paper).
+ *   lambda         : the scale factor (35 in YOCO++, section 2, key innovation 2).
  *   cache          : HOST descriptor of the destination cache.
  *   pos            : device int32 [cache->batch], first position written.
  *   cu_new         : device int32 [cache->batch + 1] prefix offsets, or NULL.
@@ -216,7 +216,7 @@ int32_t yocopp_decode_combine(const float* partials, int32_t num_parts, int64_t 
 
 /*
  * yocopp_decode_attn_static - yocopp_decode_attn without a caller workspace.
- * The paper has no counterpart: this entry point exists for callers that
+ * The pages describe no such call: this entry point exists for callers that
  * cannot allocate device memory on this path, such as a host framework that
  * owns all device memory through its own pool and gives plug-in libraries no
  * allocator, or a serving loop in which cudaMalloc's implicit device-wide
