@@ -11,11 +11,11 @@ of the bf16 probabilities it feeds, and that arguments below -126 (including the
 a wrapped exponent.
 
 This file reads the coefficients from the kernel source and replays the kernel's
-fp32 steps exactly in numpy (fp32 adds; each fused multiply-add as an exact fp64
-product plus one fp64 add, then one rounding to fp32 — the fp64 sum of an exact
-48-bit product and an fp32 addend is exact here or within an fp64 ulp, so the
-double rounding can only differ from the hardware's single rounding in ties that
-do not move the bound), then checks those properties against numpy's fp64 exp2.
+fp32 steps exactly in numpy (fp32 adds and products round correctly in numpy;
+each fused multiply-add is an exact fp64 product, an fp64 TwoSum with the
+addend, and one rounding to fp32 with ties decided by the TwoSum's error — the
+single rounding the hardware does), then checks those properties against
+numpy's fp64 exp2.  The second half replays the composition kernel's rounding.
 """
 from __future__ import annotations
 
@@ -48,8 +48,25 @@ def _cubic_coefficients():
     return [np.float32(c) for c in coef]
 
 
+def _rn32_of_sum(a64, b64):
+    """fp32 rounding (nearest, ties to even) of the exact sum a + b of two fp64 values."""
+    u = a64 + b64
+    bb = u - a64
+    e = (a64 - (u - bb)) + (b64 - bb)            # u + e == a + b exactly
+    r = u.astype(np.float32)
+    r64 = r.astype(np.float64)
+    toward = np.where(u > r64, np.float32(np.inf), np.float32(-np.inf))
+    nb = np.nextafter(r, toward)
+    nb64 = nb.astype(np.float64)
+    tie = (u != r64) & (np.abs(nb64 - u) == np.abs(u - r64))
+    past = tie & (e != 0) & (np.sign(e) == np.sign(u - r64))   # the exact sum is beyond the tie
+    return np.where(past, nb, r)
+
+
 def _fma32(a, b, c):
-    return (np.asarray(a, np.float64) * np.asarray(b, np.float64) + np.asarray(c, np.float64)).astype(np.float32)
+    """fp32 fma(a, b, c) for fp32 a, b whose product is exact in fp64 (at most 48 bits)."""
+    return _rn32_of_sum(np.asarray(a, np.float32).astype(np.float64) * np.asarray(b, np.float32).astype(np.float64),
+                        np.asarray(c, np.float32).astype(np.float64))
 
 
 def kernel_exp2(x):
@@ -117,3 +134,117 @@ def test_monotone_across_integer_boundaries():
     lo = kernel_exp2((k + 0.5 - 2 ** -12).astype(np.float32)).astype(np.float64)
     hi = kernel_exp2((k + 0.5 + 2 ** -12).astype(np.float32)).astype(np.float64)
     assert np.all(hi > lo)
+
+
+# ---------------------------------------------------------------------------
+# The composition kernel's rounding (reading 7 of the design notes: the stored
+# value is the exact composition rounded once).  Its fast path forms
+# lambda * (a1 * x1 + a2 * xi) in fp32 with error-free transformations
+# (TwoProduct by FMA, Knuth's TwoSum) and rounds the fp32 result y to bf16;
+# a y whose low 16 bits lie within 2 fp32 ulps of a bf16 rounding midpoint is
+# sent to an fp64 path that reproduces the oracle's evaluation.  The claim to
+# pin: wherever the detector lets y through, rounding y gives the same bf16 as
+# rounding the oracle's value once.  The replay below follows the kernel's
+# fp32 steps; every fused multiply-add is reproduced exactly (an fp64 product
+# that is exact, an fp64 TwoSum, and a tie decided by the TwoSum's error).
+
+LAM = 35.0
+
+
+def kernel_compose_fast(x1, xi, a1, a2, lam):
+    """The kernel's fp32 fast path, lane by lane."""
+    f = np.float32
+    x1, xi = x1.astype(f), xi.astype(f)
+    a1, a2, lam = f(a1), f(a2), f(lam)
+    p1 = (a1 * x1).astype(f)
+    n1 = _fma32(-a1, x1, p1)                     # p1 - a1*x1, exact
+    p2 = (a2 * xi).astype(f)
+    n2 = _fma32(-a2, xi, p2)
+    s = (p1 + p2).astype(f)
+    bb = (s - p1).astype(f)
+    err = ((p1 - (s - bb).astype(f)).astype(f) + (p2 - bb).astype(f)).astype(f)
+    lo = (err - (n1 + n2).astype(f)).astype(f)
+    return _fma32(lam, s, (lam * lo).astype(f))
+
+
+COMPOSE_SRC = os.path.join(ROOT, "decode_attention_yocopp_b200", "csrc", "compose_append.cuh")
+
+
+def test_replay_matches_kernel_source():
+    # the detector and the fast path's steps replayed here are the kernel's
+    src = open(COMPOSE_SRC).read()
+    assert "((__float_as_uint(y) - 0x7FFEu) & 0xFFFFu) <= 4u" in src
+    for step in ("fmul2(a1, x1)", "ffma2(na1, x1, p1)", "fadd2(p1, p2)", "fsub2(s, p1)",
+                 "fsub2(err, fadd2(n1, n2))", "ffma2(lam, s, fmul2(lam, lo))"):
+        assert step in src, step
+
+
+def _near_midpoint(y):
+    return ((y.view(np.uint32) - np.uint32(0x7FFE)) & np.uint32(0xFFFF)) <= 4
+
+
+def _rne_bf16(y):
+    b = y.view(np.uint32).astype(np.uint64)
+    return ((b + 0x7FFF + ((b >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def _bf16_values(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+@pytest.fixture(scope="module")
+def orc():
+    import oracle
+    return oracle.default()
+
+
+def _check_compose_rounding(orc, x1_bits, xi_bits, a1, a2):
+    a1, a2 = float(np.float32(a1)), float(np.float32(a2))
+    y = kernel_compose_fast(_bf16_values(x1_bits), _bf16_values(xi_bits), a1, a2, LAM)
+    exact = orc.compose(x1_bits, xi_bits, a1, a2, LAM, "bf16")
+    want = orc.round_to(exact, "bf16")
+    fast = ~_near_midpoint(y)
+    bad = fast & (_rne_bf16(y) != want)
+    assert not bad.any(), (int(bad.sum()), exact[bad][:4], y[bad][:4])
+    # the fp32 result is within two fp32 ulps of the oracle's value
+    assert np.all(np.abs(y.astype(np.float64) - exact) <= 2 * np.spacing(np.abs(y)).astype(np.float64) + 1e-300)
+    return float(1.0 - fast.mean())
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_compose_fast_path_rounds_once_on_workload_weights(orc, seed):
+    rng = np.random.default_rng(seed)
+    n = 1 << 20
+    x1 = rng.integers(0, 1 << 16, n, dtype=np.uint32).astype(np.uint16)
+    xi = rng.integers(0, 1 << 16, n, dtype=np.uint32).astype(np.uint16)
+    # finite values of moderate size (exponent field 100..154), as projections produce
+    for x in (x1, xi):
+        x &= np.uint16(0x807F)
+        x |= (rng.integers(100, 155, n).astype(np.uint16) << 7)
+    a1 = rng.uniform(-0.05, 0.05)
+    a2 = 1 / 35 + rng.uniform(-0.05, 0.05)
+    slow = _check_compose_rounding(orc, x1, xi, a1, a2)
+    assert slow < 2e-4   # the fp64 path stays rare (about 5 in 2^16)
+
+
+def test_compose_fast_path_under_cancellation(orc):
+    # a1 x1 + a2 xi with a2 = -a1 and xi next to x1: the sum cancels to a few bits
+    rng = np.random.default_rng(7)
+    n = 1 << 18
+    x1 = (rng.integers(0x3C00, 0x4200, n).astype(np.uint16)) | (rng.integers(0, 2, n).astype(np.uint16) << 15)
+    xi = (x1.astype(np.int32) + rng.integers(-3, 4, n)).astype(np.uint16)
+    for a in (0.03, 0.0417, 1 / 35):
+        _check_compose_rounding(orc, x1, xi, a, -a * (1 + 2.0 ** -20))
+
+
+@pytest.mark.parametrize("alpha", [(0.0, 1.5 / 35), (0.5 / 35, 1 / 35), (-0.75 / 35, 1.25 / 35)])
+def test_compose_detector_catches_midpoints(orc, alpha):
+    # compositions on or next to bf16 midpoints: the fast path must not decide any of them wrongly,
+    # and the detector must route the ones it cannot decide
+    mags = np.arange(0x3F80, 0x4080, dtype=np.uint32)
+    bits = np.concatenate([mags, mags | 0x8000]).astype(np.uint16)
+    rng = np.random.default_rng(11)
+    xi = np.resize(bits, 1 << 16)
+    x1 = rng.permutation(xi)
+    slow = _check_compose_rounding(orc, x1, xi, *alpha)
+    assert slow > 0.0
