@@ -137,7 +137,7 @@ def test_monotone_across_integer_boundaries():
 
 
 # ---------------------------------------------------------------------------
-# The composition kernel's rounding (reading 7 of the design notes: the stored
+# The composition kernel's rounding (the stored
 # value is the exact composition rounded once).  Its fast path forms
 # lambda * (a1 * x1 + a2 * xi) in fp32 with error-free transformations
 # (TwoProduct by FMA, Knuth's TwoSum) and rounds the fp32 result y to bf16;
