@@ -50,16 +50,17 @@ def _cubic_coefficients():
 
 def _rn32_of_sum(a64, b64):
     """fp32 rounding (nearest, ties to even) of the exact sum a + b of two fp64 values."""
-    u = a64 + b64
-    bb = u - a64
-    e = (a64 - (u - bb)) + (b64 - bb)            # u + e == a + b exactly
-    r = u.astype(np.float32)
-    r64 = r.astype(np.float64)
-    toward = np.where(u > r64, np.float32(np.inf), np.float32(-np.inf))
-    nb = np.nextafter(r, toward)
-    nb64 = nb.astype(np.float64)
-    tie = (u != r64) & (np.abs(nb64 - u) == np.abs(u - r64))
-    past = tie & (e != 0) & (np.sign(e) == np.sign(u - r64))   # the exact sum is beyond the tie
+    with np.errstate(invalid="ignore", over="ignore"):   # infinite terms: no tie to decide
+        u = a64 + b64
+        bb = u - a64
+        e = (a64 - (u - bb)) + (b64 - bb)            # u + e == a + b exactly
+        r = u.astype(np.float32)
+        r64 = r.astype(np.float64)
+        toward = np.where(u > r64, np.float32(np.inf), np.float32(-np.inf))
+        nb = np.nextafter(r, toward)
+        nb64 = nb.astype(np.float64)
+        tie = (u != r64) & (np.abs(nb64 - u) == np.abs(u - r64))
+        past = tie & (e != 0) & (np.sign(e) == np.sign(u - r64))   # the exact sum is beyond the tie
     return np.where(past, nb, r)
 
 
@@ -248,3 +249,94 @@ def test_compose_detector_catches_midpoints(orc, alpha):
     x1 = rng.permutation(xi)
     slow = _check_compose_rounding(orc, x1, xi, *alpha)
     assert slow > 0.0
+
+
+# ---------------------------------------------------------------------------
+# The causal prefill kernel's softmax, replayed on the host: per 128-key tile
+# S = q K^T in fp32, a reference maximum moved only when the tile's maximum
+# passes it by more than 8 (then l and O are rescaled), x = s * qscale - m in
+# one fp32 FMA, P = 2^x from the hardware exponential or, for one key pair in
+# four, the cubic above, P rounded to bf16, l the fp32 sum of those bf16
+# values, O += P V in fp32, out = O * (1 / l) rounded to bf16.  Checked against
+# the oracle's causal attention at the bf16 attention tolerance: the method
+# itself (bf16 probabilities against a lazily moved maximum) meets the bar,
+# whatever the order of the hardware's fp32 accumulations.
+
+LOG2E = 1.4426950408889634
+SLACK = np.float32(8.0)
+
+
+def _bf16_round_f32(x):
+    return _bf16_values(_rne_bf16(np.ascontiguousarray(x, np.float32)))
+
+
+def kernel_prefill_rows(q_bits, k_bits, v_bits, p0, scale):
+    """Output bits [n][d] of the kernel's arithmetic for query rows at positions p0 .. p0 + n - 1."""
+    q = _bf16_values(q_bits)
+    K = _bf16_values(k_bits)
+    V = _bf16_values(v_bits)
+    n, d = q.shape
+    qscale = np.float32(np.float32(scale) * np.float32(LOG2E))
+    out = np.empty((n, d), np.uint16)
+    poly = np.array([((k % 64) // 2) % 4 == 3 for k in range(128)])
+    rescales = 0
+    for r0 in range(0, n, 128):                          # one CTA's query tile
+        rows = slice(r0, min(r0 + 128, n))
+        qpos = p0 + np.arange(r0, rows.stop)
+        m_ref = np.full(len(qpos), -np.inf, np.float32)
+        l = np.zeros(len(qpos), np.float32)
+        O = np.zeros((len(qpos), d), np.float32)
+        ntk = int(qpos[-1]) // 128 + 1
+        for t in range(ntk):
+            keys = np.arange(t * 128, t * 128 + 128)
+            Kt = np.zeros((128, d), np.float32)
+            Vt = np.zeros((128, d), np.float32)
+            have = keys[keys < K.shape[0]]
+            Kt[:len(have)] = K[have]
+            Vt[:len(have)] = V[have]
+            S = (q[rows] @ Kt.T).astype(np.float32)
+            S[keys[None, :] > qpos[:, None]] = -np.inf
+            mx = S.max(axis=1)
+            m_new = np.maximum(m_ref, (mx * qscale).astype(np.float32))
+            up = m_new > (m_ref + SLACK).astype(np.float32)
+            corr = np.where(up, np.exp2((m_ref - m_new).astype(np.float32)), np.float32(1)).astype(np.float32)
+            rescales += int(np.count_nonzero(up & (t > 0)))
+            l = (l * corr).astype(np.float32)
+            O = (O * corr[:, None]).astype(np.float32)
+            m_ref = np.where(up, m_new, m_ref).astype(np.float32)
+            nm = np.where(np.isneginf(m_ref), np.float32(0), -m_ref).astype(np.float32)
+            x = _fma32(S, np.broadcast_to(qscale, S.shape), np.broadcast_to(nm[:, None], S.shape))
+            with np.errstate(over="ignore", invalid="ignore"):
+                P = np.where(poly[None, :], kernel_exp2(x), np.exp2(x).astype(np.float32))
+            Pb = _bf16_round_f32(P)
+            l = (l + Pb.sum(axis=1, dtype=np.float32)).astype(np.float32)
+            O = (O + Pb @ Vt).astype(np.float32)
+        inv = np.where(l > 0, (np.float32(1) / l).astype(np.float32), np.float32(0))
+        out[rows] = _rne_bf16((O * inv[:, None]).astype(np.float32))
+    return out, rescales
+
+
+def _composed_cache(orc, rng, T, d, value_scale=1.0):
+    def bf16(x):
+        return orc.round_to(np.asarray(x, np.float64), "bf16")
+    a1, a2 = float(np.float32(rng.uniform(-0.05, 0.05))), float(np.float32(1 / 35 + rng.uniform(-0.05, 0.05)))
+    k1, ki, v1, vi = (bf16(rng.standard_normal((T, d)) * value_scale) for _ in range(4))
+    K = orc.round_to(orc.compose(k1, ki, a1, a2, LAM, "bf16"), "bf16")
+    V = orc.round_to(orc.compose(v1, vi, a1, a2, LAM, "bf16"), "bf16")
+    return K, V
+
+
+@pytest.mark.parametrize("p0,n,qmul", [(0, 512, 1.0), (777, 300, 1.0), (0, 384, 6.0), (1000, 200, 6.0)])
+def test_prefill_softmax_replay_within_tolerance(orc, p0, n, qmul):
+    import gpu_util
+    rng = np.random.default_rng(p0 * 31 + n)
+    d = 128
+    T = p0 + n
+    K, V = _composed_cache(orc, rng, T, d)
+    q_bits = orc.round_to(rng.standard_normal((n, d)) * qmul, "bf16")
+    scale = 1.0 / np.sqrt(d)
+    got, rescales = kernel_prefill_rows(q_bits, K, V, p0, scale)
+    ref = orc.causal_attention(_bf16_values(q_bits).astype(np.float64), K, V, "bf16", scale, p0)
+    gpu_util.assert_attention(got, ref, "bf16", orc, what=f"replay p0={p0} n={n} qmul={qmul}")
+    if qmul > 1:
+        assert rescales > 0   # sharper rows move their reference maximum after the first tile
