@@ -17,7 +17,8 @@ import torch
 
 import gen
 import oracle
-from gpu_util import assert_attention, fill_sentinel, np_storage, random_block_table, scatter_rows, to_device
+from gpu_util import (assert_attention, bf16_p_spread, fill_sentinel, np_storage, random_block_table, scatter_rows,
+                      to_device)
 from oracle import model
 
 pytestmark = pytest.mark.gpu
@@ -99,7 +100,8 @@ def run_case(y, orc, *, hkv, G, nq, pos=None, capacity=None, uniform=None, key_s
         for h in range(hq):
             g = h // G
             ref = orc.causal_attention(qf[rows, h], K[b, g], V[b, g], "bf16", sc, p0=p0[b])
-            assert_attention(got[rows, h], ref, "bf16", orc, what=f"b{b} h{h}")
+            spread = bf16_p_spread(qf[rows, h], K[b, g], V[b, g], ref, sc, p0[b] + 1 + np.arange(nq[b]))
+            assert_attention(got[rows, h], ref, "bf16", orc, what=f"b{b} h{h}", p_spread=spread)
     return got
 
 
@@ -205,6 +207,12 @@ def test_out_of_capacity_is_reported(y, orc):
 # end to end: raw K/V -> yocopp_compose_append -> yocopp_prefill_attn
 # ---------------------------------------------------------------------------
 
+def _spread(w, layer, b, h, rows, kv, ref):
+    """The bf16-probability error scale of these prefill rows (token t sees keys 0..t)."""
+    q = model.prefill_queries(w, layer, b, rows)[:, h, :]
+    return bf16_p_spread(q, kv[0], kv[1], ref, 1.0 / math.sqrt(w.d), np.asarray(rows) + 1)
+
+
 def _e2e(y, orc, w, layer, rows_per_seq=None, seed=0):
     """Compose layer ``layer``'s prefill tokens into its cache, run its prefill
     attention, compare (all rows, or a sample of rows per sequence)."""
@@ -247,7 +255,8 @@ def _e2e(y, orc, w, layer, rows_per_seq=None, seed=0):
             kv = (model.composed_seq(orc, w, layer, "K", b, g)[:n], model.composed_seq(orc, w, layer, "V", b, g)[:n])
             for h in range(g * w.group, (g + 1) * w.group):
                 ref = model.prefill_self_rows(orc, w, layer, b, h, rows, kv=kv)
-                assert_attention(got_b[:, h], ref, "bf16", orc, what=f"{w.name} layer {layer} b{b} h{h}")
+                assert_attention(got_b[:, h], ref, "bf16", orc, what=f"{w.name} layer {layer} b{b} h{h}",
+                                 p_spread=_spread(w, layer, b, h, rows, kv, ref))
 
 
 def test_e2e_small_ragged(y, orc):
@@ -311,4 +320,5 @@ def _e2e_sampled_sequences(y, orc, w, layer, seqs, rows_per_seq):
             kv = (model.composed_seq(orc, w, layer, "K", b, g)[:n], model.composed_seq(orc, w, layer, "V", b, g)[:n])
             for h in range(g * w.group, (g + 1) * w.group):
                 ref = model.prefill_self_rows(orc, w, layer, b, h, rows, kv=kv)
-                assert_attention(got_b[:, h], ref, "bf16", orc, what=f"{w.name} b{b} h{h}")
+                assert_attention(got_b[:, h], ref, "bf16", orc, what=f"{w.name} b{b} h{h}",
+                                 p_spread=_spread(w, layer, b, h, rows, kv, ref))

@@ -337,6 +337,8 @@ def test_prefill_softmax_replay_within_tolerance(orc, p0, n, qmul):
     scale = 1.0 / np.sqrt(d)
     got, rescales = kernel_prefill_rows(q_bits, K, V, p0, scale)
     ref = orc.causal_attention(_bf16_values(q_bits).astype(np.float64), K, V, "bf16", scale, p0)
-    gpu_util.assert_attention(got, ref, "bf16", orc, what=f"replay p0={p0} n={n} qmul={qmul}")
+    spread = gpu_util.bf16_p_spread(_bf16_values(q_bits).astype(np.float64), K, V, ref, scale,
+                                    p0 + 1 + np.arange(n))
+    gpu_util.assert_attention(got, ref, "bf16", orc, what=f"replay p0={p0} n={n} qmul={qmul}", p_spread=spread)
     if qmul > 1:
         assert rescales > 0   # sharper rows move their reference maximum after the first tile
