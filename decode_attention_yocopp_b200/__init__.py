@@ -31,7 +31,7 @@ EXPORTS = ("yocopp_compose_append", "yocopp_decode_attn_workspace_size", "yocopp
            "yocopp_get_device_status", "yocopp_status_string", "yocopp_version",
            "yocopp_testing_set_decode_fault", "yocopp_decode_attn_static", "yocopp_decode_attn_partial",
            "yocopp_decode_combine", "yocopp_decode_attn_fused", "yocopp_set_decode_kernel",
-           "yocopp_prefill_attn")
+           "yocopp_prefill_attn", "yocopp_prefill_compose_attn_workspace_size", "yocopp_prefill_compose_attn")
 
 
 class yocopp_cache(ctypes.Structure):
@@ -90,6 +90,12 @@ def load(path: Optional[str] = None):
     lib.yocopp_prefill_attn.restype = I32
     lib.yocopp_prefill_attn.argtypes = [V, ctypes.POINTER(yocopp_cache), V, V, I32, I64, I32, V, I32,
                                         ctypes.c_float, V]
+    lib.yocopp_prefill_compose_attn_workspace_size.restype = I64
+    lib.yocopp_prefill_compose_attn_workspace_size.argtypes = [ctypes.POINTER(yocopp_cache), I32]
+    lib.yocopp_prefill_compose_attn.restype = I32
+    lib.yocopp_prefill_compose_attn.argtypes = [V, V, V, V, ctypes.POINTER(ctypes.c_float), ctypes.c_float, V,
+                                                ctypes.POINTER(yocopp_cache), V, V, I32, I64, I32, V, I32,
+                                                ctypes.c_float, V, I64, V]
     if path is None:
         _lib = lib
     return lib
@@ -253,6 +259,30 @@ def yocopp_prefill_attn(q, cache: yocopp_cache, out, pos=None, cu_q=None, n_unif
     _check("yocopp_prefill_attn", rc)
 
 
+def yocopp_prefill_compose_attn_workspace_size(cache: yocopp_cache, max_q: int) -> int:
+    n = load().yocopp_prefill_compose_attn_workspace_size(ctypes.byref(cache), int(max_q))
+    if n < 0:
+        raise YocoppError("yocopp_prefill_compose_attn_workspace_size", n)
+    return int(n)
+
+
+def yocopp_prefill_compose_attn(K1, V1, Ki, Vi, alpha, lam: float, q, cache: yocopp_cache, out, workspace,
+                                pos=None, cu_q=None, n_uniform: int = 0, total_q: Optional[int] = None,
+                                max_q: int = 0, num_q_heads: Optional[int] = None, scale: float = 0.0,
+                                stream=None) -> None:
+    """Compose the prefill rows (raw K1/V1/Ki/Vi packed like q) into the cache and run
+    the causal prefill attention over them, in one launch."""
+    hq = q.shape[1] if num_q_heads is None else num_q_heads
+    if total_q is None:
+        total_q = q.shape[0]
+    a = (ctypes.c_float * 4)(*[float(x) for x in alpha])
+    rc = load().yocopp_prefill_compose_attn(_ptr(K1), _ptr(V1), _ptr(Ki), _ptr(Vi), a, float(lam), _ptr(q),
+                                            ctypes.byref(cache), _ptr(pos), _ptr(cu_q), int(n_uniform), int(total_q),
+                                            int(max_q), _ptr(out), int(hq), float(scale), _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("yocopp_prefill_compose_attn", rc)
+
+
 STATIC_SCRATCH_BYTES = 4 << 20  # size of the library's fixed scratch array (include/yocopp.h)
 
 
@@ -273,7 +303,11 @@ def yocopp_testing_set_decode_fault(drop_tile: int = -1, wait_limit_ns: int = 2_
 
 
 def alloc_workspace(cache: yocopp_cache, num_q_heads: int, device=None):
-    """A zero-filled torch byte tensor large enough (and 256-byte aligned) for yocopp_decode_attn."""
+    """A zero-filled torch byte tensor large enough (and 256-byte aligned) for yocopp_decode_attn.
+
+    It can be reused without clearing by later calls of any batch and lengths that keep the
+    query-group size and head_dim (and pass the whole tensor); another group size or
+    head_dim needs a fresh (or re-zeroed) workspace."""
     import torch
     n = yocopp_decode_attn_workspace_size(cache, num_q_heads)
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")

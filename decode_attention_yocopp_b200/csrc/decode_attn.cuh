@@ -49,6 +49,7 @@ struct DecodeParams {
     float qscale;                // softmax scale * log2(e)
     int32_t batch, hkv, hq, capacity, block_size, mbps, num_blocks, boxr;
     int32_t num_ctas;
+    int32_t seg_units;           // split plan: tiles' worth of work a segment's flush costs
     int32_t drop_tile;           // testing: a tile whose load is never issued (-1: none)
     uint64_t wait_limit_ns;
     float* part_out;             // non-null: write unnormalised [batch][hq][D + 2] (o, m, l) instead of out
@@ -155,6 +156,61 @@ __device__ void tile_prefix(const DecodeParams& p, int* s_ts, int* s_warp) {
     __syncthreads();
 }
 
+// Split plan.  The tiles of all (sequence, kv-head) planes are flattened in
+// (b, g, tile) order, and plane P = b * hkv + g is preceded by `seg` extra
+// units: what closing a segment (flushing a partial, arriving, perhaps
+// merging) costs a CTA, in tiles.  CTA c takes the tiles whose units fall in
+// [c * unit, (c + 1) * unit), unit = ceil((tiles + seg * planes) / CTAs), so a
+// CTA that closes more segments streams fewer tiles and the CTAs finish
+// together.  unit_of(t) = t + seg * (P(t) + 1) is increasing in t.
+struct SplitPlan {
+    int total;  // tiles
+    int unit;   // units per CTA (>= 1)
+    int seg;    // units per plane start
+};
+
+__device__ __forceinline__ SplitPlan make_plan(const DecodeParams& p, const int* s_ts, int seg) {
+    SplitPlan sp;
+    sp.total = s_ts[p.batch];
+    sp.seg = seg;
+    const int64_t units = int64_t(sp.total) + int64_t(seg) * p.batch * p.hkv;
+    sp.unit = int((units + p.num_ctas - 1) / p.num_ctas);
+    if (sp.unit < 1) sp.unit = 1;
+    return sp;
+}
+
+// The first tile whose unit is >= u (sp.total if none): binary search for the
+// last plane starting at or before u, then the offset inside it.
+__device__ __forceinline__ int plan_tile_at(const DecodeParams& p, const int* s_ts, const SplitPlan& sp, int64_t u) {
+    const int planes = p.batch * p.hkv;
+    if (u >= int64_t(sp.total) + int64_t(sp.seg) * planes) return sp.total;
+    auto first_tile = [&](int P) {  // first tile of plane P
+        const int b = P / p.hkv, g = P - b * p.hkv;
+        return s_ts[b] + g * ((s_ts[b + 1] - s_ts[b]) / p.hkv);
+    };
+    int lo = 0, hi = planes;  // start unit of plane lo <= u < start unit of plane hi
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (int64_t(first_tile(mid)) + int64_t(sp.seg) * mid <= u) lo = mid; else hi = mid;
+    }
+    const int f = first_tile(lo);
+    const int64_t into = u - (int64_t(f) + int64_t(sp.seg) * (lo + 1));  // units past its cost units
+    const int t = into > 0 ? int(f + into) : f;
+    return min(t, sp.total);
+}
+
+// The CTA whose range holds tile t of plane P.
+__device__ __forceinline__ int plan_cta_of(const SplitPlan& sp, int t, int P) {
+    return int((int64_t(t) + int64_t(sp.seg) * (P + 1)) / sp.unit);
+}
+
+// This CTA's tile range [start, end): lanes 0 and 1 search, the warp shares.
+__device__ __forceinline__ int2 plan_range(const DecodeParams& p, const int* s_ts, const SplitPlan& sp, int lane) {
+    int v = 0;
+    if (lane < 2) v = plan_tile_at(p, s_ts, sp, int64_t(blockIdx.x + lane) * sp.unit);
+    return make_int2(__shfl_sync(0xffffffffu, v, 0), __shfl_sync(0xffffffffu, v, 1));
+}
+
 template <typename T, int D, int G, int W, int STAGES, bool FUSED = false>
 struct DecodeSmem {
     using S = DecodeShape<D, T, FUSED>;
@@ -162,7 +218,7 @@ struct DecodeSmem {
     static constexpr size_t up16(size_t x) { return (x + 15) & ~size_t(15); }
     static constexpr size_t kStages = size_t(STAGES) * S::STAGE_BYTES;      // 1024-aligned ring
     static constexpr size_t kBars = kStages;                                 // full[S], empty[S], sync
-    static constexpr size_t kMeta = up16(kBars + (2 * STAGES + 1) * sizeof(uint64_t));
+    static constexpr size_t kMeta = up16(kBars + (2 * STAGES + 2) * sizeof(uint64_t));  // + sync, merge
     static constexpr size_t kP = up16(kMeta + STAGES * sizeof(TileMeta));
     static constexpr size_t kMergeM = up16(kP + size_t(W) * TPW * G * sizeof(float2));
     static constexpr size_t kMergeL = up16(kMergeM + size_t(W) * G * sizeof(float));
@@ -440,15 +496,28 @@ struct ConsumerWarp {
     }
 };
 
+// Shared memory the last CTA of a plane may stage that plane's partial value
+// sums in (the tile ring, free once the CTA has consumed its last tile), with
+// an mbarrier for the bulk copy; buf == nullptr: no staging.
+struct MergeStage {
+    uint8_t* buf;
+    uint32_t bytes;
+    uint64_t* bar;
+};
+
 // Merge the partials of one (sequence, kv-head) plane written by CTAs c0..c1
 // (slots plane + cta) and write the group's outputs.  Run by the W consumer
 // warps of the last CTA to arrive.  One parallel pass stages every part's
 // maximum and sum in shared memory (the probability and warp-merge areas,
 // free at this point); weights e^{m_s - M} are formed once per (part, head);
-// then each thread accumulates 4 channels with 16-byte loads.
+// then each thread accumulates 4 channels.  With a staging area large enough,
+// the parts' value sums (contiguous slots) come in with one bulk copy issued
+// first, so that the whole merge costs one round trip to L2 for them instead
+// of one per few parts.
 template <typename T, int D, int G, int W, typename Sync>
 __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c0, int c1, int64_t out_row0,
-                                            float* scratch, int scratch_floats, Sync& sync, int tid) {
+                                            float* scratch, int scratch_floats, Sync& sync, int tid,
+                                            const MergeStage* stage) {
     constexpr int NT = W * 32;
     const int nparts = c1 - c0 + 1;
     const int cap = (scratch_floats - 2 * G) / (2 * G);  // parts that fit the staging area
@@ -470,6 +539,13 @@ __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c
             emit<T, D>(p, out_row0 + h, c, M, Ls, O);
         }
         return true;
+    }
+    const uint32_t obytes = uint32_t(nparts) * G * D * 4;
+    const bool staged = stage != nullptr && stage->buf != nullptr && obytes <= stage->bytes;
+    if (staged && tid == 0) {
+        fence_proxy_async_global();  // the parts were written (and acquired) through the generic proxy
+        mbar_arrive_expect_tx(stage->bar, obytes);
+        bulk_load(stage->buf, po, obytes, stage->bar);
     }
     float* wts = scratch;                   // [part][G]: maxima, then weights
     float* lss = scratch + cap * G;         // [part][G]: sums of exponentials
@@ -493,12 +569,18 @@ __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c
         Mh[G + tid] = Ls;
     }
     ok = sync() && ok;
+    if (staged) {
+        // every thread waits (bounded) for the bulk copy; a warp continues only if all its lanes saw it
+        ok = __all_sync(0xffffffffu, mbar_wait(stage->bar, 0, p.wait_limit_ns)) && ok;
+        if (!ok) return false;
+        po = reinterpret_cast<const float4*>(stage->buf);
+    }
     for (int q4 = tid; q4 < G * D / 4; q4 += NT) {
         const int h = (q4 * 4) / D;
         float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
         for (int s2 = 0; s2 < nparts; ++s2) {
-            const float4 o = __ldcg(po + int64_t(s2) * (G * D / 4) + q4);
+            const float4 o = staged ? po[int64_t(s2) * (G * D / 4) + q4] : __ldcg(po + int64_t(s2) * (G * D / 4) + q4);
             const float f = wts[s2 * G + h];
             O.x += f * o.x; O.y += f * o.y; O.z += f * o.z; O.w += f * o.w;
         }
@@ -527,10 +609,10 @@ __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c
 // the W consumer warps (ctid = consumer thread index).  False on a timed-out
 // rendezvous.
 template <typename T, int D, int G, int W, typename Sync>
-__device__ __forceinline__ bool flush_segment(const DecodeParams& p, const TileMeta& mt, int ctid, int tpc,
+__device__ __forceinline__ bool flush_segment(const DecodeParams& p, const TileMeta& mt, int ctid, const SplitPlan& sp,
                                               const int* s_ts, float* mg_m, float* mg_l, float* mg_o, float* scratch,
                                               int scratch_floats, Sync& consumer_sync, int& s_last,
-                                              unsigned long long epoch) {
+                                              unsigned long long epoch, const MergeStage* stage = nullptr) {
     if (!consumer_sync()) return false;
     const int bg = mt.b * p.hkv + mt.g;
     const int slot = bg + int(blockIdx.x);
@@ -565,7 +647,7 @@ __device__ __forceinline__ bool flush_segment(const DecodeParams& p, const TileM
         if (!consumer_sync()) return false;
         const int nt = ntiles_of(mt.len, mt.pad);  // pad carries the kernel's tile size
         const int first = s_ts[mt.b] + mt.g * nt;
-        const int c0 = first / tpc, c1 = (first + nt - 1) / tpc;
+        const int c0 = plan_cta_of(sp, first, bg), c1 = plan_cta_of(sp, first + nt - 1, bg);
         if (ctid == 0) {
             const unsigned arrived = arrive_plane(p.ws_cnt + bg, epoch);
             if (arrived == 0) record_status(YOCOPP_EWORKSPACE);
@@ -575,7 +657,7 @@ __device__ __forceinline__ bool flush_segment(const DecodeParams& p, const TileM
         if (!consumer_sync()) return false;
         if (s_last) {
             if (!merge_plane<T, D, G, W>(p, bg, c0, c1, int64_t(mt.b) * p.hq + mt.g * G, scratch, scratch_floats,
-                                         consumer_sync, ctid))
+                                         consumer_sync, ctid, stage))
                 return false;
         }
     }
@@ -600,6 +682,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(base + L::kBars);
     uint64_t* empty_bar = full_bar + STAGES;
     uint64_t* sync_bar = empty_bar + STAGES;  // consumer warps' merge rendezvous
+    uint64_t* merge_bar = sync_bar + 1;       // the final merge's bulk copy
     TileMeta* meta = reinterpret_cast<TileMeta*>(base + L::kMeta);
     float* p_s = reinterpret_cast<float*>(base + L::kP);
     float* mg_m = reinterpret_cast<float*>(base + L::kMergeM);
@@ -615,6 +698,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             mbar_init(&empty_bar[s], W);
         }
         mbar_init(sync_bar, W);
+        mbar_init(merge_bar, 1);
         fence_mbar_init();
         s_abort = 0;
         s_cdone = 0;
@@ -634,10 +718,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             emit<T, D>(p, int64_t(b) * p.hq + idx / D, idx % D, NEG_INF_F, 0.f, 0.f);
     }
 
-    const int total = s_ts[p.batch];
-    const int tpc = (total + p.num_ctas - 1) / p.num_ctas;
-    const int start = min(int(blockIdx.x) * tpc, total);
-    const int end = min(start + tpc, total);
+    const SplitPlan sp = make_plan(p, s_ts, p.seg_units);
+    const int2 range = plan_range(p, s_ts, sp, lane);
+    const int start = range.x, end = range.y;
     if (start >= end) return;
 
     if (warp == W) {
@@ -812,9 +895,11 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         if (mt.flags & kLast) {
             // ---- end of segment: merge the warps' states, emit output or a partial
             cw.stash(mg_m, mg_l, mg_o);
-            if (!flush_segment<T, D, G, W>(p, mt, tid, tpc, s_ts, mg_m, mg_l, mg_o, p_s,
+            // at the CTA's last tile the ring is free: a final merge may stage partials there
+            const MergeStage ring{stage_mem, uint32_t(L::kStages), merge_bar};
+            if (!flush_segment<T, D, G, W>(p, mt, tid, sp, s_ts, mg_m, mg_l, mg_o, p_s,
                                            int((L::kTileStart - L::kP) / sizeof(float)), consumer_sync, s_last,
-                                           epoch)) {
+                                           epoch, t == end - 1 ? &ring : nullptr)) {
                 record_status(YOCOPP_ETIMEOUT);
                 s_abort = 1;
                 break;

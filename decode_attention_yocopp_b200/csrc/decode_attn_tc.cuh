@@ -46,8 +46,8 @@ struct TcSmem {
     using S = TcShape;
     static constexpr size_t up16(size_t x) { return (x + 15) & ~size_t(15); }
     static constexpr size_t kStages = size_t(STAGES) * S::STAGE_BYTES;
-    static constexpr size_t kBars = kStages;  // full[S], empty[S], sfull[2], sempty[2], sync
-    static constexpr size_t kTmem = up16(kBars + (2 * STAGES + 5) * sizeof(uint64_t));
+    static constexpr size_t kBars = kStages;  // full[S], empty[S], sfull[2], sempty[2], sync, merge
+    static constexpr size_t kTmem = up16(kBars + (2 * STAGES + 6) * sizeof(uint64_t));
     static constexpr size_t kMeta = up16(kTmem + 16);
     static constexpr size_t kP = up16(kMeta + STAGES * sizeof(TileMeta));
     static constexpr size_t kMergeM = up16(kP + size_t(S::W) * S::TPW * G * sizeof(float2));
@@ -199,6 +199,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     __shared__ volatile int s_abort;
     __shared__ int s_cdone;
     __shared__ int s_last;
+    // the call's epoch: taken by an otherwise idle lane of the MMA warp (its atomics are
+    // round trips to L2) while the first tiles load; the consumers need it at their first flush
+    __shared__ unsigned long long s_epoch;
+    __shared__ volatile int s_epoch_ready;
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stage_mem = base;
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(base + L::kBars);
@@ -206,6 +210,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     uint64_t* sfull_bar = empty_bar + STAGES;   // accumulator b holds a finished score tile
     uint64_t* sempty_bar = sfull_bar + 2;       // accumulator b has been read
     uint64_t* sync_bar = sempty_bar + 2;        // consumer warps' merge rendezvous
+    uint64_t* merge_bar = sync_bar + 1;         // the final merge's bulk copy
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L::kTmem);
     TileMeta* meta = reinterpret_cast<TileMeta*>(base + L::kMeta);
     float* p_s = reinterpret_cast<float*>(base + L::kP);
@@ -226,35 +231,36 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             mbar_init(&sempty_bar[b], W);
         }
         mbar_init(sync_bar, W);
+        mbar_init(merge_bar, 1);
         fence_mbar_init();
         s_abort = 0;
         s_cdone = 0;
+        s_epoch_ready = 0;
     }
-    griddep_wait();
-    griddep_launch_dependents();
-    __shared__ unsigned long long s_epoch;
-    if (tid == 0) s_epoch = join_call(p.ws_gen, gridDim.x);
-    tile_prefix<TILE>(p, s_ts, s_warp);  // ends with __syncthreads()
-    const unsigned long long epoch = s_epoch;
-    for (int b = blockIdx.x; b < p.batch; b += p.num_ctas) {
-        if (s_ts[b + 1] != s_ts[b]) continue;
-        for (int idx = tid; idx < p.hq * S::D; idx += blockDim.x)
-            emit<__nv_bfloat16, S::D>(p, int64_t(b) * p.hq + idx / S::D, idx % S::D, NEG_INF_F, 0.f, 0.f);
-    }
-    const int total = s_ts[p.batch];
-    const int tpc = (total + p.num_ctas - 1) / p.num_ctas;
-    const int start = min(int(blockIdx.x) * tpc, total);
-    const int end = min(start + tpc, total);
-    if (start >= end) return;
-
+    // tensor memory needs no input: take it while the previous kernel may still run
     if (warp == 1) {
         tmem_alloc(tmem_slot, S::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
-    __syncthreads();
+    griddep_wait();
+    griddep_launch_dependents();
+    tile_prefix<TILE>(p, s_ts, s_warp);  // ends with __syncthreads()
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    for (int b = blockIdx.x; b < p.batch; b += p.num_ctas) {
+        if (s_ts[b + 1] != s_ts[b]) continue;
+        for (int idx = tid; idx < p.hq * S::D; idx += blockDim.x)
+            emit<__nv_bfloat16, S::D>(p, int64_t(b) * p.hq + idx / S::D, idx % S::D, NEG_INF_F, 0.f, 0.f);
+    }
+    const SplitPlan sp = make_plan(p, s_ts, p.seg_units);
+    const int2 range = plan_range(p, s_ts, sp, lane);
+    const int start = range.x, end = range.y;
+    if (start >= end) {
+        if (tid == 0) (void)join_call(p.ws_gen, gridDim.x);  // every CTA joins the call
+        if (warp == 1) tmem_dealloc(tmem, S::TMEM_COLS);
+        return;
+    }
 
     if (warp == 0) {
         // ------------------------------------------------------------------ producer
@@ -380,6 +386,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     if (warp == 1) {
         // ------------------------------------------------------------- MMA issuer
         int last_it[2] = {-1, -1};
+        if (lane == 1) {
+            s_epoch = join_call(p.ws_gen, gridDim.x);
+            __threadfence_block();
+            s_epoch_ready = 1;
+        }
         if (lane == 0) {
             int it = 0;
             for (int t = start; t < end; ++t, ++it) {
@@ -436,6 +447,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         return ok;
     };
 
+    unsigned long long epoch = 0;  // epochs start at 1
     int it = 0;
     for (int t = start; t < end; ++t, ++it) {
         const int stage = it % STAGES;
@@ -466,10 +478,25 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         if (lane == 0) mbar_arrive(&empty_bar[stage]);
 
         if (mt.flags & kLast) {
+            if (epoch == 0) {  // first flush: the epoch was taken long ago
+                const uint64_t t0 = globaltimer_ns();
+                while (!s_epoch_ready && globaltimer_ns() - t0 <= p.wait_limit_ns) __nanosleep(32);
+                if (!__all_sync(0xffffffffu, s_epoch_ready != 0)) {
+                    record_status(YOCOPP_ETIMEOUT);
+                    s_abort = 1;
+                    break;
+                }
+                __threadfence_block();
+                epoch = s_epoch;
+            }
             cw.stash(mg_m, mg_l, mg_o);
-            if (!flush_segment<__nv_bfloat16, S::D, G, W>(p, mt, ctid, tpc, s_ts, mg_m, mg_l, mg_o, p_s,
+            // at the CTA's last tile the ring is free (every load and product that used it
+            // has completed): a final merge may stage partials there
+            const MergeStage ring{stage_mem, uint32_t(L::kStages), merge_bar};
+            if (!flush_segment<__nv_bfloat16, S::D, G, W>(p, mt, ctid, sp, s_ts, mg_m, mg_l, mg_o, p_s,
                                                           int((L::kTileStart - L::kP) / sizeof(float)),
-                                                          consumer_sync, s_last, epoch)) {
+                                                          consumer_sync, s_last, epoch,
+                                                          t == end - 1 ? &ring : nullptr)) {
                 record_status(YOCOPP_ETIMEOUT);
                 s_abort = 1;
                 break;

@@ -44,6 +44,7 @@
 // copies and products in flight, frees the tensor memory and returns.
 #pragma once
 
+#include "compose_append.cuh"
 #include "decode_attn.cuh"
 
 namespace yocopp {
@@ -62,6 +63,19 @@ struct PrefillParams {
     float qscale;           // softmax scale * log2(e)
     uint64_t wait_limit_ns;
     int32_t drop_k_tile;    // testing: K tile whose load CTA 0 never issues (-1: none)
+    // fused composition (prefill_tc_kernel<true> only): raw rows of layer 1 and of
+    // this layer, packed like q ([total_q][hkv][128] bf16), the weights, the cache
+    // planes the composed rows go to, and the call generation and per-(sequence,
+    // query tile) flags in the caller's workspace
+    const uint8_t* k1;
+    const uint8_t* v1;
+    const uint8_t* ki;
+    const uint8_t* vi;
+    uint8_t* ck;
+    uint8_t* cv;
+    float ak1, ak2, av1, av2, lam;
+    unsigned long long* ws_gen;  // [0] last finished call's generation, [1] call arrivals
+    unsigned long long* flags;   // [batch][q_tiles]: generation of the call that composed the tile
 };
 
 struct PfShape {
@@ -87,10 +101,14 @@ static_assert(PfShape::SMEM <= 232448 - 16, "prefill shared memory");
 
 // 2^x on the FMA pipe for two arguments at once (fp32x2 arithmetic), for
 // x <= 2^22 (x below -126 is taken as -126, whose result, at most 2^-125.5,
-// is nothing next to the row's largest term 1): x = j + f with j = round(x),
+// is nothing next to the row's largest term 1; a causally masked key's -inf
+// therefore gets a weight of at most 2^-125.5 here, where MUFU gives 0: the
+// row sum is at least 2^-8, so such a key moves the output by at most 2^-117
+// of its value row, which the fp32 sums cannot even represent, and its value
+// row lies inside the window, so it is finite): x = j + f with j = round(x),
 // f in [-1/2, 1/2] (Cody and Waite's range reduction, with the round done by
 // adding 1.5 * 2^23), 2^f from a cubic fitted here to the relative error on
-// [-1/2, 1/2] (max 7.5e-5, far below the 2^-9 of the bf16 probabilities it
+// [-1/2, 1/2] (max 7.5e-5, far below the 2^-8 rounding of the bf16 probabilities it
 // feeds), and 2^j added to the exponent field.  The exponential unit does 16
 // results per clock per SM, one tile's worth in the time the tensor cores take
 // for it; moving a quarter of them here keeps it off the critical path.
@@ -130,6 +148,136 @@ __device__ __forceinline__ float2 add_bf16x2(float2 acc, uint32_t w) {
 // a quarter of the exponentials on the FMA pipe, the rest on MUFU).
 __device__ __forceinline__ constexpr bool poly_pair(int e) { return (e & 3) == 3; }
 
+// Fused composition: compose query tile jt's rows of sequence b (every KV head)
+// from the raw layer-1 and layer-i rows with the arithmetic of
+// yocopp_compose_append (so the stored bits are the same) and write them to
+// their cache positions p_b + jt * 128 + r.  The four input streams are
+// contiguous here (the tile's (token, head) rows), so lane 0 of warp 0 stages
+// them into shared memory with 1-D bulk copies, 64 rows (16 KB) of each
+// stream per stage, three stages deep; warps 1..9 compose from shared memory
+// and store the cache rows.  All threads of the CTA call it.
+__device__ __forceinline__ void prefill_compose_tile(const PrefillParams& p, int b, int jt, int tid, uint8_t* smem) {
+    using S = PfShape;
+    constexpr int SROWS = 64, STAGES = 3, SBYTES = SROWS * 256;  // per stream and stage
+    constexpr int NC = S::THREADS - 32;                           // composing threads
+    static_assert(STAGES * 4 * SBYTES <= S::BAR_OFF, "composition stages fit below the barriers");
+    int qrow0, nq;
+    if (p.cu_q) {
+        qrow0 = __ldg(p.cu_q + b);
+        nq = __ldg(p.cu_q + b + 1) - qrow0;
+    } else {
+        qrow0 = b * p.n_uniform;
+        nq = p.n_uniform;
+    }
+    const int p0 = p.pos ? __ldg(p.pos + b) : 0;
+    // an invalid sequence is reported by its attention CTAs
+    if (nq < 0 || p0 < 0 || int64_t(p0) + nq > p.capacity || nq > p.q_tiles * S::TQ) return;
+    const int r0 = jt * S::TQ;
+    const int n = min(S::TQ, nq - r0);
+    if (n <= 0) return;
+    const int rows = n * p.hkv;                                   // the tile's (token, head) rows
+    const int nsb = (rows + SROWS - 1) / SROWS;
+    const int64_t in0 = (int64_t(qrow0) + r0) * p.hkv * 256;      // byte offset of its first input row
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+    uint64_t* empty = full + STAGES;
+    const int warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], NC / 32);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int sb = 0; sb < nsb; ++sb) {
+                const int st = sb % STAGES;
+                if (!mbar_wait(&empty[st], ((sb / STAGES) & 1) ^ 1, p.wait_limit_ns)) {
+                    record_status(YOCOPP_ETIMEOUT);
+                    break;
+                }
+                const int r = sb * SROWS;
+                const uint32_t bytes = uint32_t(min(SROWS, rows - r)) * 256u;
+                mbar_arrive_expect_tx(&full[st], 4u * bytes);
+                uint8_t* dst = smem + st * 4 * SBYTES;
+                const int64_t off = in0 + int64_t(r) * 256;
+                bulk_load(dst, p.k1 + off, bytes, &full[st]);
+                bulk_load(dst + SBYTES, p.ki + off, bytes, &full[st]);
+                bulk_load(dst + 2 * SBYTES, p.v1 + off, bytes, &full[st]);
+                bulk_load(dst + 3 * SBYTES, p.vi + off, bytes, &full[st]);
+                issued = sb + 1;
+            }
+            // the copies still in flight land before the CTA may exit
+            for (int sb = issued > STAGES ? issued - STAGES : 0; sb < issued; ++sb)
+                (void)mbar_wait(&full[sb % STAGES], (sb / STAGES) & 1, p.wait_limit_ns);
+        }
+        return;
+    }
+    const ComposeCoef ck = make_coef(p.ak1, p.ak2, p.lam);
+    const ComposeCoef cv = make_coef(p.av1, p.av2, p.lam);
+    const int ctid = tid - 32;
+    for (int sb = 0; sb < nsb; ++sb) {
+        const int st = sb % STAGES;
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (sb / STAGES) & 1, p.wait_limit_ns))) {
+            record_status(YOCOPP_ETIMEOUT);
+            break;
+        }
+        const int r = sb * SROWS;
+        const int nrow = min(SROWS, rows - r);
+        const uint8_t* src = smem + st * 4 * SBYTES;
+        for (int i = ctid; i < nrow * 16; i += NC) {
+            const int lr = i >> 4, c = i & 15;
+            const int row = r + lr;
+            const int tok = row / p.hkv, h = row % p.hkv;
+            const int position = p0 + r0 + tok;
+            int64_t dst;
+            if (p.block_table == nullptr) {
+                dst = ((int64_t(b) * p.hkv + h) * p.capacity + position) * 256;
+            } else {
+                const int blk = __ldg(p.block_table + int64_t(b) * p.mbps + position / p.block_size);
+                if (blk < 0 || blk >= p.num_blocks) {
+                    record_status(YOCOPP_EDEVICE_CHECK);
+                    continue;
+                }
+                dst = ((int64_t(blk) * p.hkv + h) * p.block_size + position % p.block_size) * 256;
+            }
+            const int so = lr * 256 + c * 16;
+            const uint4 k1 = *reinterpret_cast<const uint4*>(src + so);
+            const uint4 ki = *reinterpret_cast<const uint4*>(src + SBYTES + so);
+            const uint4 v1 = *reinterpret_cast<const uint4*>(src + 2 * SBYTES + so);
+            const uint4 vi = *reinterpret_cast<const uint4*>(src + 3 * SBYTES + so);
+            st_global(p.ck + dst + c * 16, compose_chunk<__nv_bfloat16>(k1, ki, ck));
+            st_global(p.cv + dst + c * 16, compose_chunk<__nv_bfloat16>(v1, vi, cv));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+    }
+}
+
+// Wait (bounded) until the flag holds this call's generation.
+__device__ __forceinline__ bool wait_flag(const unsigned long long* f, unsigned long long epoch, uint64_t limit_ns) {
+    if (ld_acquire_gpu(f) == epoch) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_gpu(f) != epoch) {
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+        __nanosleep(128);
+    }
+    return true;
+}
+
+// FUSED: the grid also composes the rows it attends over.  Per sequence b there
+// are q_tiles composition CTAs (one per 128-row query tile, every KV head) and
+// the attention CTAs of the unfused kernel; the composition CTAs of sequence
+// b + 1 are placed before the attention CTAs of sequence b, so they run one
+// sequence ahead.  A composition CTA publishes its tile's flag (this call's
+// generation, release) after its stores; an attention CTA's loaders wait
+// (acquire, bounded) for the flags of every query tile whose rows a key tile
+// holds before loading it.  Blocks are dispatched in index order, so every
+// flag an attention CTA waits for belongs to a CTA that is already running or
+// done, and no CTA waits on a later one.
+template <bool FUSED>
 __global__ void __launch_bounds__(PfShape::THREADS, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
@@ -146,8 +294,41 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const int G = p.hq / p.hkv;
     const int units = G / p.heads_per_cta;                         // CTAs per (sequence, KV head, tile)
     const int per_plane = p.q_tiles * units;
-    const int plane = int(blockIdx.x) / per_plane;                 // b * hkv + g
-    const int rem = int(blockIdx.x) % per_plane;
+    int bidx = int(blockIdx.x);                                    // index in the attention order
+    unsigned long long epoch = 0;
+    if constexpr (FUSED) {
+        __shared__ unsigned long long s_ep;
+        if (tid == 0) s_ep = join_call(p.ws_gen, gridDim.x);
+        __syncthreads();
+        epoch = s_ep;
+        const int per_attn = p.hkv * per_plane;
+        int cb = -1, cjt = 0;
+        if (bidx < p.q_tiles) {
+            cb = 0;
+            cjt = bidx;
+        } else {
+            const int i = bidx - p.q_tiles;
+            const int sq = i / (p.q_tiles + per_attn), r = i % (p.q_tiles + per_attn);
+            if (sq + 1 < p.batch && r < p.q_tiles) {
+                cb = sq + 1;
+                cjt = r;
+            } else {
+                bidx = sq * per_attn + (sq + 1 < p.batch ? r - p.q_tiles : r);
+            }
+        }
+        if (cb >= 0) {
+            prefill_compose_tile(
+                p, cb, cjt, tid,
+                reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023)));
+            fence_proxy_async_global();
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) st_release_gpu(p.flags + int64_t(cb) * p.q_tiles + cjt, epoch);
+            return;
+        }
+    }
+    const int plane = bidx / per_plane;                            // b * hkv + g
+    const int rem = bidx % per_plane;
     const int jt = p.q_tiles - 1 - rem / units;
     const int b = plane / p.hkv;
     const int g = plane % p.hkv;
@@ -239,11 +420,26 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             }
             const int plane_row = (b * p.hkv + g) * p.capacity;
             const int nsb = S::TK / p.boxr;  // boxes of boxr rows per tile (one per cache block)
+            int composed_upto = -1;          // FUSED: query tiles of this call seen composed
             for (int t = 0; t < ntk; ++t) {
                 const int slot = t & 1;
                 if (s_abort || !mbar_wait(&empty[slot], ((t >> 1) & 1) ^ 1, p.wait_limit_ns)) {
                     ok = false;
                     break;
+                }
+                if constexpr (FUSED) {
+                    // this call's positions in the key tile come from query tiles .. c_hi
+                    const int hi = min(t * S::TK + S::TK, kv_len) - 1;
+                    if (hi >= p0) {
+                        const int c_hi = (hi - p0) / S::TQ;
+                        while (ok && composed_upto < c_hi) {
+                            ok = wait_flag(p.flags + int64_t(b) * p.q_tiles + composed_upto + 1, epoch,
+                                           p.wait_limit_ns);
+                            if (ok) ++composed_upto;
+                        }
+                        if (!ok) break;
+                        fence_proxy_async_global();
+                    }
                 }
                 if (kl && t == p.drop_k_tile && blockIdx.x == 0) continue;  // failure injection (tests)
                 // the tile's rows: one 128-row box (contiguous), or one box per cache block;

@@ -2,6 +2,7 @@
 // planning and kernel launches for the YOCO++ compose/append and the shared-
 // cache decode attention.  One translation unit holds every kernel so the
 // device status word is a single symbol.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -20,9 +21,12 @@ constexpr int kMaxBatch = 8192;
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
 
-int g_test_drop_tile = -1;
-int g_decode_kernel = 0;  // 0 / 2: tensor-core scores where supported, 1: CUDA-core scores
-uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
+// Process-wide settings written by the setters below and read at every launch;
+// atomics, since launches may run on other host threads (relaxed: each value
+// stands alone).
+std::atomic<int> g_test_drop_tile{-1};
+std::atomic<int> g_decode_kernel{0};  // 0 / 2: tensor-core scores where supported, 1: CUDA-core scores
+std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -128,6 +132,10 @@ int32_t launch_compose(ComposeParams& p, cudaStream_t st) {
 #ifndef YOCOPP_DECODE_CTAS_PER_SM
 #define YOCOPP_DECODE_CTAS_PER_SM 2
 #endif
+// Split plan: what closing a segment (flush, arrival, merge) costs a CTA, in tiles.
+#ifndef YOCOPP_DECODE_SEG_UNITS
+#define YOCOPP_DECODE_SEG_UNITS 3
+#endif
 
 struct DecodeLaunch {
     int w, stages, tile, ctas_per_sm;
@@ -227,9 +235,10 @@ bool encode_q3d(CUtensorMap* map, const void* base, int heads, int head_dim, int
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <bool FUSED>
 int32_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p,
                        int64_t grid, cudaStream_t st) {
-    auto kern = prefill_tc_kernel;
+    auto kern = prefill_tc_kernel<FUSED>;
     static bool attr_set[kMaxDevices] = {false};
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices) return YOCOPP_ECUDA;
@@ -251,22 +260,41 @@ int32_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     return cuda_status(cudaLaunchKernelEx(&lc, kern, tq, tk, tv, p));
 }
 
+// Decode workspace: a 256-byte header (call generation + call arrivals), the
+// split partials m [slots][G], l [slots][G], o [slots][G][D] (fp32) from offset
+// 256 upwards, and the per-plane arrival counters at the END of the buffer.
+// Slots are sized for the larger of the two decode grids (plane + CTA index),
+// so the partials' extent depends only on (planes, G, D) and grows with the
+// plane count.  Counters of a call therefore never land on bytes an earlier
+// call with the same G and D (and the same buffer size) used for partials:
+// a call with more planes has its counters lower down, but its partials, and
+// every earlier call's, end below them.
 struct WorkspaceLayout {
-    size_t gen, cnt, m, l, o, total;
+    size_t gen, m, l, o, partial_end, cnt;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
-WorkspaceLayout workspace_layout(int batch, int hkv, int G, int D, int num_ctas) {
-    const size_t slots = size_t(num_ctas) + size_t(batch) * hkv;
+// planes = batch * hkv; max_ctas = the larger decode grid; buf_bytes = the
+// buffer's size; cnt_words = counter words reserved at its end (>= planes).
+WorkspaceLayout workspace_layout(size_t planes, int G, int D, int max_ctas, size_t buf_bytes, size_t cnt_words) {
+    const size_t slots = size_t(max_ctas) + planes;
     WorkspaceLayout w;
-    w.gen = 0;                      // header: generation word + call-arrival word
-    w.cnt = 256;
-    w.m = w.cnt + up256(size_t(batch) * hkv * sizeof(unsigned long long));
+    w.gen = 0;
+    w.m = 256;
     w.l = w.m + up256(slots * G * sizeof(float));
     w.o = w.l + up256(slots * G * sizeof(float));
-    w.total = w.o + up256(slots * G * D * sizeof(float));
+    w.partial_end = w.o + up256(slots * G * D * sizeof(float));
+    const size_t cnt_bytes = up256(cnt_words * sizeof(unsigned long long));
+    const size_t top = buf_bytes & ~size_t(255);
+    w.cnt = top >= cnt_bytes ? top - cnt_bytes : 0;
     return w;
+}
+
+// Bytes yocopp_decode_attn_workspace_size reports: partials plus the counters right after.
+size_t workspace_bytes_needed(size_t planes, int G, int D, int max_ctas) {
+    const WorkspaceLayout w = workspace_layout(planes, G, D, max_ctas, 0, 0);
+    return w.partial_end + up256(planes * sizeof(unsigned long long));
 }
 
 int32_t check_decode_shape(const yocopp_cache* cache, int32_t num_q_heads, int* G) {
@@ -290,6 +318,7 @@ int32_t check_decode_shape(const yocopp_cache* cache, int32_t num_q_heads, int* 
 // image, so callers that cannot allocate device memory still get a workspace.
 // Every device that loads the library holds it until the process exits.
 constexpr size_t kStaticScratchBytes = size_t(4) << 20;  // 4 MiB
+constexpr size_t kStaticCounterWords = 8192;              // planes (batch x kv heads) a static call may have
 static __device__ __align__(256) uint8_t g_decode_scratch[kStaticScratchBytes];
 
 namespace {
@@ -343,14 +372,14 @@ int32_t yocopp_get_device_status(int32_t reset) {
 
 int32_t yocopp_set_decode_kernel(int32_t which) {
     if (which < 0 || which > 2) return YOCOPP_EINVAL;
-    g_decode_kernel = which;
+    g_decode_kernel.store(which, std::memory_order_relaxed);
     return YOCOPP_OK;
 }
 
 int32_t yocopp_testing_set_decode_fault(int32_t drop_tile, int64_t wait_limit_ns) {
     if (wait_limit_ns <= 0) return YOCOPP_EINVAL;
-    g_test_drop_tile = drop_tile < 0 ? -1 : drop_tile;
-    g_wait_limit_ns = uint64_t(wait_limit_ns);
+    g_test_drop_tile.store(drop_tile < 0 ? -1 : drop_tile, std::memory_order_relaxed);
+    g_wait_limit_ns.store(uint64_t(wait_limit_ns), std::memory_order_relaxed);
     return YOCOPP_OK;
 }
 
@@ -408,8 +437,8 @@ int64_t yocopp_decode_attn_workspace_size(const yocopp_cache* cache, int32_t num
     if (rc != YOCOPP_OK) return rc;
     const int sms = sm_count(current_device());
     if (sms <= 0) return YOCOPP_ECUDA;
-    return int64_t(workspace_layout(cache->batch, cache->num_kv_heads, G, cache->head_dim,
-                                    sms * YOCOPP_DECODE_CTAS_PER_SM).total);
+    return int64_t(workspace_bytes_needed(size_t(cache->batch) * cache->num_kv_heads, G, cache->head_dim,
+                                          sms * YOCOPP_DECODE_CTAS_PER_SM));
 }
 
 // fused != nullptr: the read-time composition variant; `cache` holds raw K_i, V_i,
@@ -419,9 +448,12 @@ struct FusedArgs {
     float coef[4];
 };
 
+// cnt_words: arrival-counter words reserved at the end of the workspace (0: one per
+// plane of this call, the caller-workspace layout).
 static int32_t decode_attn_impl(const void* q, const yocopp_cache* cache, const int32_t* seq_lens, void* out,
                                 float* part_out, int32_t num_q_heads, float scale, void* workspace,
-                                int64_t workspace_bytes, void* stream, const FusedArgs* fused = nullptr) {
+                                int64_t workspace_bytes, void* stream, const FusedArgs* fused = nullptr,
+                                size_t cnt_words = 0) {
     int G = 0;
     int32_t rc = check_decode_shape(cache, num_q_heads, &G);
     if (rc != YOCOPP_OK) return rc;
@@ -444,12 +476,16 @@ static int32_t decode_attn_impl(const void* q, const yocopp_cache* cache, const 
     if (sms <= 0) return YOCOPP_ECUDA;
     // tensor-core scores: bf16, head_dim 128, no read-time composition, block size >= 16, and the
     // batch's tile table fits next to the 3-stage ring
-    const bool use_tc = g_decode_kernel != 1 && fused == nullptr && cache->dtype == YOCOPP_BF16 &&
+    const bool use_tc = g_decode_kernel.load(std::memory_order_relaxed) != 1 && fused == nullptr && cache->dtype == YOCOPP_BF16 &&
                         cache->head_dim == 128 && TcSmem<4, 3>::bytes(cache->batch) <= 232448 - 1024;
     const int num_ctas = use_tc ? sms : sms * YOCOPP_DECODE_CTAS_PER_SM;
-    const WorkspaceLayout wl = workspace_layout(cache->batch, cache->num_kv_heads, G, cache->head_dim, num_ctas);
-    if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < int64_t(wl.total))
+    const size_t planes = size_t(cache->batch) * cache->num_kv_heads;
+    if (cnt_words == 0) cnt_words = planes;
+    if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes <= 0 || cnt_words < planes)
         return YOCOPP_EWORKSPACE;
+    const WorkspaceLayout wl = workspace_layout(planes, G, cache->head_dim, sms * YOCOPP_DECODE_CTAS_PER_SM,
+                                                size_t(workspace_bytes), cnt_words);
+    if (wl.cnt < wl.partial_end) return YOCOPP_EWORKSPACE;
 
     const int D = cache->head_dim;
     const int tile = use_tc ? TcShape::TILE : ((D * elem_bytes(cache->dtype)) <= 256 ? 64 : 32) / (fused != nullptr ? 2 : 1);
@@ -492,8 +528,9 @@ static int32_t decode_attn_impl(const void* q, const yocopp_cache* cache, const 
     p.num_blocks = paged ? cache->num_blocks : 0;
     p.boxr = boxr;
     p.num_ctas = num_ctas;
-    p.drop_tile = g_test_drop_tile;
-    p.wait_limit_ns = g_wait_limit_ns;
+    p.seg_units = YOCOPP_DECODE_SEG_UNITS;
+    p.drop_tile = g_test_drop_tile.load(std::memory_order_relaxed);
+    p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
     p.part_out = part_out;
     p.fa1k = fused ? fused->coef[0] : 0.f;
     p.fa2k = fused ? fused->coef[1] : 0.f;
@@ -587,22 +624,40 @@ int32_t yocopp_decode_combine(const float* partials, int32_t num_parts, int64_t 
 
 // Decode attention whose workspace is the library's own static device array
 // (no allocation anywhere).  Argument meaning as yocopp_decode_attn.
+// The counter region sits at a fixed place (the array's last kStaticCounterWords
+// words) whatever the shape, so no call's partials ever overlap another call's
+// counters.
 int32_t yocopp_decode_attn_static(const void* q, const yocopp_cache* cache, const int32_t* seq_lens, void* out,
                                   int32_t num_q_heads, float scale, void* stream) {
     const int64_t need = yocopp_decode_attn_workspace_size(cache, num_q_heads);
     if (need < 0) return int32_t(need);
-    if (need > int64_t(kStaticScratchBytes)) return YOCOPP_EWORKSPACE;
+    if (out == nullptr) return YOCOPP_EINVAL;
+    if (int64_t(cache->batch) * cache->num_kv_heads > int64_t(kStaticCounterWords)) return YOCOPP_EWORKSPACE;
     void* scratch = static_scratch_ptr(current_device());
     if (scratch == nullptr) return YOCOPP_ECUDA;
-    return yocopp_decode_attn(q, cache, seq_lens, out, num_q_heads, scale, scratch,
-                              int64_t(kStaticScratchBytes), stream);
+    // too large a shape fails the partials-below-counters check with YOCOPP_EWORKSPACE
+    return decode_attn_impl(q, cache, seq_lens, out, nullptr, num_q_heads, scale, scratch,
+                            int64_t(kStaticScratchBytes), stream, nullptr, kStaticCounterWords);
 }
 
 // Causal prefill attention of a self-decoder layer over its own cache
-// (tcgen05 for both products).  Argument meaning in yocopp.h.
-int32_t yocopp_prefill_attn(const void* q, const yocopp_cache* cache, const int32_t* pos, const int32_t* cu_q,
-                            int32_t n_uniform, int64_t total_q, int32_t max_q, void* out, int32_t num_q_heads,
-                            float scale, void* stream) {
+// (tcgen05 for both products); with `fused`, the same launch first composes
+// the rows it attends over from raw inputs.  Argument meaning in yocopp.h.
+struct PrefillFused {
+    const void *k1, *v1, *ki, *vi;
+    const float* alpha;
+    float lambda;
+    void* workspace;
+    int64_t workspace_bytes;
+};
+
+static int64_t prefill_fused_ws_bytes(int32_t batch, int q_tiles) {
+    return int64_t(256) + ((int64_t(batch) * q_tiles * 8 + 255) & ~int64_t(255));
+}
+
+static int32_t prefill_attn_impl(const void* q, const yocopp_cache* cache, const int32_t* pos, const int32_t* cu_q,
+                                 int32_t n_uniform, int64_t total_q, int32_t max_q, void* out, int32_t num_q_heads,
+                                 float scale, void* stream, const PrefillFused* fused) {
     const int32_t rc = check_cache(cache);
     if (rc != YOCOPP_OK) return rc;
     if (cache->dtype != YOCOPP_BF16) return YOCOPP_EDTYPE;
@@ -623,17 +678,31 @@ int32_t yocopp_prefill_attn(const void* q, const yocopp_cache* cache, const int3
                                : int64_t(cache->batch) * cache->num_kv_heads * cache->capacity;
     if (rows + PfShape::TK >= (int64_t(1) << 31)) return YOCOPP_EINVAL;  // tile row coordinates stay 32-bit
     const int boxr = paged ? (cache->block_size < PfShape::TK ? cache->block_size : PfShape::TK) : PfShape::TK;
-    if (total_q == 0 || max_q == 0) return YOCOPP_OK;
     const int q_tiles = (max_q + PfShape::TQ - 1) / PfShape::TQ;
+    if (fused != nullptr) {
+        if (fused->alpha == nullptr || !std::isfinite(fused->lambda) || !std::isfinite(fused->alpha[0]) ||
+            !std::isfinite(fused->alpha[1]) || !std::isfinite(fused->alpha[2]) || !std::isfinite(fused->alpha[3]))
+            return YOCOPP_EINVAL;
+        if (total_q > 0 && (fused->k1 == nullptr || fused->v1 == nullptr || fused->ki == nullptr ||
+                            fused->vi == nullptr || !aligned(fused->k1, 16) || !aligned(fused->v1, 16) ||
+                            !aligned(fused->ki, 16) || !aligned(fused->vi, 16)))
+            return YOCOPP_EINVAL;
+        if (fused->workspace == nullptr || !aligned(fused->workspace, 256) ||
+            fused->workspace_bytes < prefill_fused_ws_bytes(cache->batch, q_tiles))
+            return YOCOPP_EWORKSPACE;
+    }
+    if (total_q == 0 || max_q == 0) return YOCOPP_OK;
     const int heads_per_cta = (num_q_heads / cache->num_kv_heads) % 2 == 0 ? 2 : 1;
-    const int64_t grid = int64_t(q_tiles) * cache->batch * (num_q_heads / heads_per_cta);
+    int64_t grid = int64_t(q_tiles) * cache->batch * (num_q_heads / heads_per_cta);
+    if (fused != nullptr) grid += int64_t(q_tiles) * cache->batch;  // the composition CTAs
     if (grid >= (int64_t(1) << 31)) return YOCOPP_EINVAL;
+    if (fused != nullptr && grid >= (int64_t(1) << 20)) return YOCOPP_EINVAL;  // the call-arrival count field
     alignas(64) CUtensorMap tq, tk, tv;
     if (!encode_q3d(&tq, q, num_q_heads, 128, total_q, PfShape::TQ) ||
         !encode_rows(&tk, cache->k, YOCOPP_BF16, 128, rows, boxr) ||
         !encode_rows(&tv, cache->v, YOCOPP_BF16, 128, rows, boxr))
         return YOCOPP_ECUDA;
-    PrefillParams p;
+    PrefillParams p = {};
     p.out = static_cast<uint8_t*>(out);
     p.pos = pos;
     p.cu_q = cu_q;
@@ -651,9 +720,54 @@ int32_t yocopp_prefill_attn(const void* q, const yocopp_cache* cache, const int3
     p.heads_per_cta = heads_per_cta;
     const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(128.f);
     p.qscale = sc * 1.4426950408889634f;
-    p.wait_limit_ns = g_wait_limit_ns;
-    p.drop_k_tile = g_test_drop_tile;
-    return launch_prefill(tq, tk, tv, p, grid, static_cast<cudaStream_t>(stream));
+    p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+    p.drop_k_tile = g_test_drop_tile.load(std::memory_order_relaxed);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (fused == nullptr) return launch_prefill<false>(tq, tk, tv, p, grid, st);
+    p.k1 = static_cast<const uint8_t*>(fused->k1);
+    p.v1 = static_cast<const uint8_t*>(fused->v1);
+    p.ki = static_cast<const uint8_t*>(fused->ki);
+    p.vi = static_cast<const uint8_t*>(fused->vi);
+    p.ck = static_cast<uint8_t*>(cache->k);
+    p.cv = static_cast<uint8_t*>(cache->v);
+    p.ak1 = fused->alpha[0];
+    p.ak2 = fused->alpha[1];
+    p.av1 = fused->alpha[2];
+    p.av2 = fused->alpha[3];
+    p.lam = fused->lambda;
+    uint8_t* ws = static_cast<uint8_t*>(fused->workspace);
+    p.ws_gen = reinterpret_cast<unsigned long long*>(ws);
+    p.flags = reinterpret_cast<unsigned long long*>(ws + 256);
+    return launch_prefill<true>(tq, tk, tv, p, grid, st);
+}
+
+int32_t yocopp_prefill_attn(const void* q, const yocopp_cache* cache, const int32_t* pos, const int32_t* cu_q,
+                            int32_t n_uniform, int64_t total_q, int32_t max_q, void* out, int32_t num_q_heads,
+                            float scale, void* stream) {
+    return prefill_attn_impl(q, cache, pos, cu_q, n_uniform, total_q, max_q, out, num_q_heads, scale, stream,
+                             nullptr);
+}
+
+int64_t yocopp_prefill_compose_attn_workspace_size(const yocopp_cache* cache, int32_t max_q) {
+    if (cache == nullptr || cache->batch < 1 || cache->batch > kMaxBatch || max_q < 0) return YOCOPP_EINVAL;
+    return prefill_fused_ws_bytes(cache->batch, (max_q + PfShape::TQ - 1) / PfShape::TQ);
+}
+
+int32_t yocopp_prefill_compose_attn(const void* K1, const void* V1, const void* Ki, const void* Vi,
+                                    const float alpha[4], float lambda, const void* q, const yocopp_cache* cache,
+                                    const int32_t* pos, const int32_t* cu_q, int32_t n_uniform, int64_t total_q,
+                                    int32_t max_q, void* out, int32_t num_q_heads, float scale, void* workspace,
+                                    int64_t workspace_bytes, void* stream) {
+    PrefillFused f;
+    f.k1 = K1;
+    f.v1 = V1;
+    f.ki = Ki;
+    f.vi = Vi;
+    f.alpha = alpha;
+    f.lambda = lambda;
+    f.workspace = workspace;
+    f.workspace_bytes = workspace_bytes;
+    return prefill_attn_impl(q, cache, pos, cu_q, n_uniform, total_q, max_q, out, num_q_heads, scale, stream, &f);
 }
 
 }  // extern "C"

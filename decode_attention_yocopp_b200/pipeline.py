@@ -16,7 +16,8 @@ from typing import Dict, List, Optional, Sequence, Tuple
 
 import torch
 
-from . import (alloc_workspace, make_cache, yocopp_compose_append, yocopp_decode_attn, yocopp_prefill_attn)
+from . import (alloc_workspace, make_cache, yocopp_compose_append, yocopp_decode_attn, yocopp_prefill_attn,
+               yocopp_prefill_compose_attn, yocopp_prefill_compose_attn_workspace_size)
 
 LAMBDA = 35.0
 
@@ -89,5 +90,21 @@ class SharedKVStack:
         ``write`` has appended the same tokens (bf16, head_dim 128, contiguous or paged)."""
         yocopp_prefill_attn(q, self.desc[i], out, pos=pos, cu_q=cu_q, n_uniform=n_uniform, total_q=q.shape[0],
                             max_q=max_q, num_q_heads=self.hq, scale=scale, stream=stream)
+        return out
+
+    def prefill_write_attend(self, i: int, k1: torch.Tensor, v1: torch.Tensor, ki: torch.Tensor, vi: torch.Tensor,
+                             q: torch.Tensor, out: torch.Tensor, pos: Optional[torch.Tensor] = None,
+                             cu_q: Optional[torch.Tensor] = None, n_uniform: int = 0, max_q: int = 0,
+                             scale: float = 0.0, stream=None) -> torch.Tensor:
+        """``write`` then ``prefill_attend`` of the same prefill tokens in one launch: layer i's
+        rows composed from the raw inputs (layer 1: stored raw) and attended causally."""
+        mq = n_uniform if cu_q is None else max_q
+        need = yocopp_prefill_compose_attn_workspace_size(self.desc[i], mq)
+        ws = getattr(self, "_prefill_ws", None)
+        if ws is None or ws.numel() < need or ws.device != q.device:
+            ws = self._prefill_ws = torch.zeros(need, dtype=torch.uint8, device=q.device)
+        yocopp_prefill_compose_attn(k1, v1, ki, vi, self.layer_alpha(i), self.lam, q, self.desc[i], out, ws,
+                                    pos=pos, cu_q=cu_q, n_uniform=n_uniform, total_q=q.shape[0], max_q=max_q,
+                                    num_q_heads=self.hq, scale=scale, stream=stream)
         return out
 

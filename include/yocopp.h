@@ -125,14 +125,23 @@ int32_t yocopp_compose_append(const void* K1, const void* V1, const void* Ki, co
  * yocopp_decode_attn_workspace_size - bytes of device workspace that
  * yocopp_decode_attn needs for this cache shape and query-head count on the
  * current device (it depends on the device's SM count).  Returns a negative
- * yocopp_status on invalid arguments.  The workspace holds the per-split
- * partial softmax state (max, sum of exponentials, weighted value sum),
- * per-(sequence, kv-head) arrival counters, and a call generation that the
- * kernel itself advances (so calls captured in a CUDA graph replay
- * correctly).  Zero-fill the workspace once before its first use; after that
- * it never needs clearing, also not after a failed call.  (A workspace that
- * was never zero-filled can make a call report YOCOPP_EWORKSPACE through
- * yocopp_get_device_status.)
+ * yocopp_status on invalid arguments.  The workspace holds a call generation
+ * that the kernel itself advances (so calls captured in a CUDA graph replay
+ * correctly), the per-split partial softmax state (max, sum of exponentials,
+ * weighted value sum) from the start of the buffer upwards, and one arrival
+ * counter per (sequence, kv-head) plane at the END of the buffer
+ * (workspace_bytes as passed, rounded down to 256).
+ *
+ * Zero-fill the workspace once before its first use.  After that it never
+ * needs clearing, also not after a failed call, as long as every call on it
+ * passes the same workspace_bytes, the same query-group size (num_q_heads /
+ * num_kv_heads) and the same head_dim; batch and lengths may change freely
+ * between calls (the partials' extent only grows with the plane count, so it
+ * never reaches the counters of a call with more planes).  Zero-fill it again
+ * before using it with another group size, head_dim or workspace_bytes.  A
+ * workspace that was not zero-filled can make a call report
+ * YOCOPP_EWORKSPACE through yocopp_get_device_status and leave output rows
+ * unwritten.
  */
 int64_t yocopp_decode_attn_workspace_size(const yocopp_cache* cache, int32_t num_q_heads);
 
@@ -226,19 +235,24 @@ int32_t yocopp_decode_combine(const float* partials, int32_t num_parts, int64_t 
  * split partials and arrival counters live in a fixed 4 MiB array inside the
  * library (every device that loads the library holds it until the process
  * exits).  Nothing is allocated or freed by this call.
- *   - A shape whose workspace (yocopp_decode_attn_workspace_size) exceeds
- *     that capacity returns YOCOPP_EWORKSPACE and enqueues nothing.  At
- *     head_dim 128 and 4 query heads per KV head that is roughly
- *     batch * num_kv_heads <= 1800 on a 148-SM device.
+ *   - The array's last 64 KiB hold the arrival counters of up to 8192
+ *     (sequence, kv-head) planes at a fixed place; the split partials use the
+ *     rest.  A shape with batch * num_kv_heads > 8192, or whose partials do
+ *     not fit, returns YOCOPP_EWORKSPACE and enqueues nothing.  On a 148-SM
+ *     device at head_dim 128 that is batch * num_kv_heads <= 1688 with 4
+ *     query heads per KV head, 3673 with 2 and 7642 with 1 (partials:
+ *     (2 * 148 + batch * num_kv_heads) * G * (head_dim + 2) * 4 bytes, each of
+ *     the three arrays rounded up to 256, within 4 MiB - 64 KiB - 256).
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress with that device current); make that first call
  *     before any stream capture.
  *   - All calls on a device share the one array and it keeps the last call's
- *     contents.  It starts zero-filled when the library is loaded, and every
- *     call (also a failed one) leaves it usable by the next, so nothing ever
- *     needs clearing.  Calls whose execution overlaps on the GPU (different
- *     streams, or different host threads) race on it and give wrong results:
- *     serialise them.
+ *     contents.  It starts zero-filled when the library is loaded; since the
+ *     counters never move and the partials never reach them, every call (also
+ *     a failed one, and whatever the previous call's shape) leaves it usable
+ *     by the next, so nothing ever needs clearing.  Calls whose execution
+ *     overlaps on the GPU (different streams, or different host threads) race
+ *     on it and give wrong results: serialise them.
  */
 int32_t yocopp_decode_attn_static(const void* q, const yocopp_cache* cache, const int32_t* seq_lens,
                                   void* out, int32_t num_q_heads, float scale, void* stream);
@@ -285,6 +299,42 @@ int32_t yocopp_decode_attn_static(const void* q, const yocopp_cache* cache, cons
 int32_t yocopp_prefill_attn(const void* q, const yocopp_cache* cache, const int32_t* pos, const int32_t* cu_q,
                             int32_t n_uniform, int64_t total_q, int32_t max_q, void* out, int32_t num_q_heads,
                             float scale, void* stream);
+
+/*
+ * yocopp_prefill_compose_attn - yocopp_compose_append followed by
+ * yocopp_prefill_attn in ONE launch: the composition of the prefill rows
+ * fused with the causal attention over them (YOCO++: Enhancing YOCO with KV
+ * Residual Connections, section 2, composition equations and cache strategy;
+ * section 3: prefill is compute-bound and the composition adds only a little
+ * I/O, which here overlaps the attention's tensor-core work).  The launch
+ * holds, per sequence, one composition CTA for each 128-row query tile (all
+ * KV heads) besides the attention CTAs; the composition CTAs of sequence b+1
+ * run ahead of the attention CTAs of sequence b, and an attention CTA waits
+ * (bounded, on a flag in the workspace) until the rows of a key tile are
+ * composed before loading it.  Results equal the two calls': the cache gets
+ * the same bits as yocopp_compose_append writes and the outputs those of
+ * yocopp_prefill_attn.
+ *
+ *   K1, V1, Ki, Vi : raw rows as for yocopp_compose_append, packed like q
+ *                    ([total_q][num_kv_heads][128] bf16, rows of sequence b
+ *                    at [cu_q[b], cu_q[b+1]) or b * n_uniform ..); they are
+ *                    composed into cache positions pos[b] + j.
+ *   alpha, lambda  : as for yocopp_compose_append (HOST alpha[4]).
+ *   q ... scale    : as for yocopp_prefill_attn.
+ *   workspace      : device, >= yocopp_prefill_compose_attn_workspace_size()
+ *                    bytes, 256-byte aligned, zero-filled once before its first
+ *                    use; it never needs clearing after that (a call generation
+ *                    advanced by the kernel tags the flags), for any later
+ *                    shape.  Not shared with a concurrently running call.
+ * Positions before pos[b] must already hold composed rows, as for
+ * yocopp_prefill_attn.  A wait that runs out records YOCOPP_ETIMEOUT.
+ */
+int64_t yocopp_prefill_compose_attn_workspace_size(const yocopp_cache* cache, int32_t max_q);
+int32_t yocopp_prefill_compose_attn(const void* K1, const void* V1, const void* Ki, const void* Vi,
+                                    const float alpha[4], float lambda, const void* q, const yocopp_cache* cache,
+                                    const int32_t* pos, const int32_t* cu_q, int32_t n_uniform, int64_t total_q,
+                                    int32_t max_q, void* out, int32_t num_q_heads, float scale, void* workspace,
+                                    int64_t workspace_bytes, void* stream);
 
 /*
  * yocopp_get_device_status - the first error code recorded by a kernel on

@@ -222,3 +222,23 @@ def test_unzeroed_workspace_is_reported(y):
         y.yocopp_decode_attn(q, cache, lens, out, ws)
         assert y.yocopp_get_device_status(reset=True) == 0
         assert torch.equal(out, ref)
+
+
+def test_workspace_reused_as_plane_count_changes(y, orc):
+    # one caller workspace, zero-filled once and sized for the largest call, reused
+    # by calls whose plane counts (batch x kv heads) grow and shrink with the same
+    # group size and head_dim: the header's contract says it never needs clearing
+    from gpu_util import DecodeCase
+    rng = np.random.default_rng(5)
+    cases = [DecodeCase(51, [4096, 3000, 2500], 4, 4),
+             DecodeCase(52, [int(x) for x in rng.integers(1, 1500, size=30)], 8, 4, paged=True),
+             DecodeCase(53, [3000, 5000, 100, 2000], 8, 4),
+             DecodeCase(54, [int(x) for x in rng.integers(1, 1000, size=64)], 8, 4)]
+    need = max(y.yocopp_decode_attn_workspace_size(c.cache(y), c.hkv * c.G) for c in cases)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for i, c in enumerate(cases):
+        out = torch.full_like(c.q, float("nan"))
+        y.yocopp_decode_attn(c.q, c.cache(y), c.seq_lens, out, ws)
+        torch.cuda.synchronize()
+        assert y.yocopp_get_device_status(reset=True) == 0, f"call {i}"
+        assert_attention(np_storage(out), c.reference(orc), "bf16", orc, f"reused workspace, call {i}")
