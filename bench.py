@@ -56,6 +56,9 @@ def parse():
                     help="profiling only: compose just the last N self-decoder layers (0 = all)")
     ap.add_argument("--cross-layers", type=int, default=0,
                     help="profiling only: run just N cross-decoder layers (0 = all)")
+    ap.add_argument("--workloads", default=None,
+                    help="comma-separated further long-context workloads measured after the headline one, each "
+                         "reported under 'workloads' (default: 4,5 with the headline workload 3, else none)")
     return ap.parse_args()
 
 
@@ -325,9 +328,10 @@ class Step:
         for i in self.comp:
             s.write(i, self.kn[1], self.vn[1], self.kn[i], self.vn[i], self.posn, n_uniform=1)
         rec("t2")
+        # the cross-decoder layers back to back (no event between them, so that each launch
+        # overlaps the previous one's tail as programmatic dependent launches do in a real step)
         for l in self.cross:
             s.cross_attend(self.q[l], self.lens, self.out[l])
-            rec("attn")
         rec("t3")
 
 
@@ -355,7 +359,7 @@ def run_ours(args, rank, world, local):
     if st != 0:
         raise RuntimeError(f"device status after warm-up: {y.yocopp_status_string(st)}")
 
-    ev = {k: [] for k in ("t0", "t1", "t2", "t3", "attn")}
+    ev = {k: [] for k in ("t0", "t1", "t2", "t3")}
     clocks = Clocks(local) if rank == 0 else None
     if clocks:
         clocks.start()
@@ -373,12 +377,8 @@ def run_ours(args, rank, world, local):
     t_prefill = sum(a.elapsed_time(b) for a, b in zip(ev["t0"], ev["t1"]))
     t_dcomp = sum(a.elapsed_time(b) for a, b in zip(ev["t1"], ev["t2"]))
     t_attn = sum(a.elapsed_time(b) for a, b in zip(ev["t2"], ev["t3"]))
-    # per-layer attention launch durations (split + combine), events between layers
-    per_layer = []
-    for s_i in range(args.steps):
-        nc = len(cross_layers)
-        marks = [ev["t2"][s_i]] + ev["attn"][s_i * nc:(s_i + 1) * nc]
-        per_layer += [a.elapsed_time(b) for a, b in zip(marks[:-1], marks[1:])]
+    # average attention launch duration: the cross-decoder layers' span over their count
+    per_layer = [t_attn / (args.steps * len(cross_layers))]
 
     K = args.steps
     kv_bytes_layer = w.kv_bytes()
@@ -447,6 +447,14 @@ def run_ours(args, rank, world, local):
     status = y.yocopp_get_device_status(reset=True)
     if status != 0:
         raise RuntimeError(f"device status after timing: {y.yocopp_status_string(status)}")
+    launches = step.launches_per_step * K
+    del step
+    torch.cuda.empty_cache()
+
+    legs = None
+    leg_cfgs = args.workloads if args.workloads is not None else ("4,5" if args.config == 3 else "")
+    if leg_cfgs and not (args.compose_layers or args.cross_layers):
+        legs = [run_leg(int(c), args, rank, world, local) for c in leg_cfgs.split(",") if c.strip()]
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -477,7 +485,9 @@ def run_ours(args, rank, world, local):
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(total_max / K, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "storage": w.dtype, "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "accumulate": "f32",
+        "dtype_note": "caches, q and both tensor-core operands in the storage type; fp32 arithmetic and accumulation",
+        "data": "synthetic",
         "config": {"workload": workload, "layers": w.layers, "batch_per_gpu": w.batch, "global_batch": w.batch * world,
                    "context": w.max_len if w.uniform else "ragged", "q_heads": w.hq, "kv_heads": w.hkv,
                    "head_dim": w.d, "paged": w.paged, "parallelism": f"dp{world} (sequences per rank, no exchange)",
@@ -506,12 +516,89 @@ def run_ours(args, rank, world, local):
         "profiling_trim": bool(args.compose_layers or args.cross_layers),
         "roofline_attention": roof_attn,
         "roofline_compose": roof_comp,
-        "gpu_launches": step.launches_per_step * K,
+        "gpu_launches": launches,
         "clocks": clk,
         "e2e": e2e,
         "cpu_baseline": cpu,
+        "workloads": legs,
     }
     return line
+
+
+def run_leg(cfg, args, rank, world, local):
+    """A further workload, measured like the headline step (same steps and warm-up,
+    CUDA events on the launching stream, max over ranks) with the decode-attention
+    and compose rooflines, decode tok/s and the prefill attention beside it."""
+    import torch
+    import decode_attention_yocopp_b200 as y
+    w = rank_workload(cfg, rank)
+    step = Step(w)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    st = y.yocopp_get_device_status(reset=True)
+    if st != 0:
+        raise RuntimeError(f"{w.name}: device status after warm-up: {y.yocopp_status_string(st)}")
+    ev = {k: [] for k in ("t0", "t1", "t2", "t3")}
+    clocks = Clocks(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    for _ in range(args.steps):
+        step.run(ev)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    K, nc, ncomp = args.steps, len(step.cross), len(step.comp)
+    t_prefill = sum(a.elapsed_time(b) for a, b in zip(ev["t0"], ev["t1"]))
+    t_dcomp = sum(a.elapsed_time(b) for a, b in zip(ev["t1"], ev["t2"]))
+    t_attn = sum(a.elapsed_time(b) for a, b in zip(ev["t2"], ev["t3"]))
+    per_layer = [t_attn / (K * nc)]
+    t_attn_max = max_over_ranks(t_attn, world)
+    t_prefill_max = max_over_ranks(t_prefill, world)
+    t_decode_max = max_over_ranks(t_attn + t_dcomp, world)
+    kv_all = sum_over_ranks(w.kv_bytes() * nc * K, world)
+    comp_all = sum_over_ranks(w.compose_bytes(w.total_prefill) * ncomp * K, world)
+    tok_all = sum_over_ranks(w.batch * K, world)
+    prefill = None
+    if not args.no_prefill and w.dtype == "bf16" and w.d == 128:
+        prefill = run_prefill_attention(args, step, world)
+    status = y.yocopp_get_device_status(reset=True)
+    if status != 0:
+        raise RuntimeError(f"{w.name}: device status after timing: {y.yocopp_status_string(status)}")
+    del step
+    torch.cuda.empty_cache()
+    peak, peak_kind = hbm_peak()
+    ach_attn = w.kv_bytes() / (sum(per_layer) / len(per_layer) * 1e-3) / 1e9
+    ach_comp = w.compose_bytes(w.total_prefill) / (t_prefill / (K * ncomp) * 1e-3) / 1e9
+    dk = decode_kernel_name(w, args.decode_kernel)
+    return {
+        "workload": w.name,
+        "config": {"layers": w.layers, "batch_per_gpu": w.batch, "context": w.max_len if w.uniform else "ragged",
+                   "total_context": int(sum(w.lens)), "q_heads": w.hq, "kv_heads": w.hkv, "head_dim": w.d,
+                   "paged": w.paged, "planted_key": w.planted is not None, "storage": w.dtype},
+        "steps": K, "warmup": args.warmup,
+        "decode_attention": {"kernel": dk, "kv_read_gbs_job": round(kv_all / (t_attn_max * 1e-3) / 1e9, 1),
+                             "achieved_gbs_per_layer": round(ach_attn, 1),
+                             "ms_per_layer": round(sum(per_layer) / len(per_layer), 4),
+                             "frac_of_measured": round(ach_attn / peak, 4),
+                             "frac_of_nominal": round(ach_attn / NOMINAL_HBM_GBS, 4), "peak": peak,
+                             "peak_kind": peak_kind, "traffic": ncu_traffic(dk, w.name),
+                             "algorithmic_bytes_per_launch": w.kv_bytes()},
+        "compose": {"kernel": "compose_append_kernel (prefill size)",
+                    "gbs_job": round(comp_all / (t_prefill_max * 1e-3) / 1e9, 1),
+                    "achieved_gbs_per_launch": round(ach_comp, 1),
+                    "frac_of_measured": round(ach_comp / peak, 4),
+                    "frac_of_nominal": round(ach_comp / NOMINAL_HBM_GBS, 4),
+                    "traffic": ncu_traffic("compose_append_kernel", w.name),
+                    "algorithmic_bytes_per_launch": w.compose_bytes(w.total_prefill)},
+        "decode_tok_s": round(tok_all / (t_decode_max * 1e-3), 1),
+        "decode_compose_us_per_layer": round(1e3 * t_dcomp / (K * ncomp), 2),
+        "prefill_attention": prefill,
+        "clocks": clk,
+    }
 
 
 def tensor_peak():
@@ -558,6 +645,7 @@ def run_prefill_attention(args, step, world):
     burst, sustained, kind = tensor_peak()
     ach = flops / (sum(per) / K * 1e-3) / 1e12
     job = sum_over_ranks(flops * K, world) / (t_max * 1e-3) / 1e12
+    fused = run_prefill_fused(step, q, out, K, kw, world)
     del q, out
     return {"kernel": "prefill_tc_kernel", "what": "causal attention of one self-decoder layer's prefill tokens "
                                                    "over its own composed cache (bf16, tcgen05 for q.K and P.V)",
@@ -568,7 +656,46 @@ def run_prefill_attention(args, step, world):
                          "frac": round(ach / burst, 4), "peak_kind": f"{kind} bf16 burst",
                          "frac_of_sustained": round(ach / sustained, 4),
                          "algorithmic_flops_per_launch": flops,
-                         "traffic": ncu_traffic("prefill_tc_kernel", w.name)}}
+                         "traffic": ncu_traffic("prefill_tc_kernel", w.name)},
+            "compose_fused": fused}
+
+
+def run_prefill_fused(step, q, out, K, kw, world):
+    """The shared layer's prefill rows composed and attended: two launches
+    (yocopp_compose_append, then yocopp_prefill_attn) against one fused launch
+    (yocopp_prefill_compose_attn), each timed per pass with CUDA events."""
+    import torch
+    w, s = step.w, step.stack
+    L = w.shared_layer
+    pos0 = step.pos0
+
+    def two():
+        if step.cu is None:
+            s.write(L, step.kp[1], step.vp[1], step.kp[L], step.vp[L], pos0, n_uniform=w.lens[0] - 1)
+        else:
+            s.write(L, step.kp[1], step.vp[1], step.kp[L], step.vp[L], pos0, cu_new=step.cu)
+        s.prefill_attend(L, q, out, pos=pos0, **kw)
+
+    def one():
+        s.prefill_write_attend(L, step.kp[1], step.vp[1], step.kp[L], step.vp[L], q, out, pos=pos0, **kw)
+
+    res = {}
+    for name, fn in (("two_launches", two), ("fused", one)):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        barrier(world)
+        marks = [_event()]
+        for _ in range(K):
+            fn()
+            marks.append(_event())
+        torch.cuda.synchronize()
+        per = [a.elapsed_time(b) for a, b in zip(marks[:-1], marks[1:])]
+        res[name + "_ms"] = round(max_over_ranks(sum(per), world) / K, 4)
+    res["fused_speedup"] = round(res["two_launches_ms"] / res["fused_ms"], 4)
+    res["what"] = ("composition of the shared layer's prefill rows + their causal attention: "
+                   "yocopp_compose_append then yocopp_prefill_attn, against yocopp_prefill_compose_attn")
+    return res
 
 
 def run_e2e(args, step, world):
