@@ -13,7 +13,11 @@ Reported (one JSON line from rank 0):
   value      decode-attention KV-read GB/s: algorithmic KV bytes of all
              cross-decoder layers / their measured time (whole job, all ranks)
   compose_gbs, decode_tok_s, roofline (dominant kernel), e2e (same metric
-  through the C ABI with host buffers), clocks, cpu_baseline (the oracle).
+  through the C ABI with host buffers), clocks, cpu_baseline (the oracle),
+  prefill_attention (the causal prefill attention, and the fused composition +
+  prefill launch against the two separate launches), and, after the headline
+  32 x 8192 workload, the 131072-token and the ragged paged workloads measured
+  the same way under "workloads".
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
 workload and prints the same line with "impl": "reference".
 """

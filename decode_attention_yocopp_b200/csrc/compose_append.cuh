@@ -152,14 +152,15 @@ __device__ __forceinline__ int64_t cache_row_offset(const ComposeParams& p, int 
 }
 
 // Launch shape (compile-time; the defaults are the measured best on B200).
-// One 1024-thread CTA per SM, one chunk per thread per iteration: the grid is
-// exactly resident (no second-wave tail), and each iteration of the grid-
-// stride loop sweeps 148 x 1024 consecutive chunks of every stream.
+// One 1024-thread CTA per SM, two chunks of every stream in flight per thread
+// (measured +3% over one at 32 x 8192, the same on the ragged paged batch): the
+// grid is exactly resident (no second-wave tail), and each iteration of the
+// grid-stride loop sweeps 2 x 148 x 1024 consecutive chunks of every stream.
 #ifndef YOCOPP_COMPOSE_THREADS
 #define YOCOPP_COMPOSE_THREADS 1024
 #endif
 #ifndef YOCOPP_COMPOSE_UNROLL
-#define YOCOPP_COMPOSE_UNROLL 1
+#define YOCOPP_COMPOSE_UNROLL 2
 #endif
 #ifndef YOCOPP_COMPOSE_CTAS_PER_SM
 #define YOCOPP_COMPOSE_CTAS_PER_SM 1

@@ -235,8 +235,9 @@ struct DecodeSmem {
 // header[0] for the next call.  Every CTA arrives right after reading, before
 // any work that could time out, so each call advances the epoch exactly once;
 // the epoch lives on the device, so a captured CUDA graph replays correctly.
-__device__ __forceinline__ unsigned long long join_call(unsigned long long* hdr, unsigned num_ctas) {
-    const unsigned long long epoch = __ldcg(hdr) + 1ull;
+// The arrival half of join_call, for a CTA that read the epoch (header[0] + 1)
+// earlier: any time after that read will do.
+__device__ __forceinline__ void arrive_call(unsigned long long* hdr, unsigned long long epoch, unsigned num_ctas) {
     __threadfence();
     atomicMax(hdr + 1, epoch << 20);
     const unsigned long long old = atomicAdd(hdr + 1, 1ull);
@@ -244,6 +245,11 @@ __device__ __forceinline__ unsigned long long join_call(unsigned long long* hdr,
         __threadfence();
         atomicMax(hdr, epoch);
     }
+}
+
+__device__ __forceinline__ unsigned long long join_call(unsigned long long* hdr, unsigned num_ctas) {
+    const unsigned long long epoch = __ldcg(hdr) + 1ull;
+    arrive_call(hdr, epoch, num_ctas);
     return epoch;
 }
 
@@ -514,17 +520,33 @@ struct MergeStage {
 // the parts' value sums (contiguous slots) come in with one bulk copy issued
 // first, so that the whole merge costs one round trip to L2 for them instead
 // of one per few parts.
+// own >= 0: part `own` (this CTA's) was not published; its state is the W
+// consumer warps' stash (mg_m, mg_l: [W][G], mg_o: [W][G][D]) and is merged
+// from there.
+template <int D, int G, int W>
+__device__ __forceinline__ void own_state(const float* mg_m, const float* mg_l, int h, float& M, float& Ls) {
+    M = NEG_INF_F;
+#pragma unroll
+    for (int w2 = 0; w2 < W; ++w2) M = fmaxf(M, mg_m[w2 * G + h]);
+    Ls = 0.f;
+    if (M != NEG_INF_F) {
+#pragma unroll
+        for (int w2 = 0; w2 < W; ++w2) Ls += exp2f(mg_m[w2 * G + h] - M) * mg_l[w2 * G + h];
+    }
+}
+
 template <typename T, int D, int G, int W, typename Sync>
 __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c0, int c1, int64_t out_row0,
                                             float* scratch, int scratch_floats, Sync& sync, int tid,
-                                            const MergeStage* stage) {
+                                            const MergeStage* stage, int own = -1, const float* mg_m = nullptr,
+                                            const float* mg_l = nullptr, const float* mg_o = nullptr) {
     constexpr int NT = W * 32;
     const int nparts = c1 - c0 + 1;
     const int cap = (scratch_floats - 2 * G) / (2 * G);  // parts that fit the staging area
     const float* pm = p.ws_m + int64_t(bg + c0) * G;
     const float* pl = p.ws_l + int64_t(bg + c0) * G;
     const float4* po = reinterpret_cast<const float4*>(p.ws_o + int64_t(bg + c0) * G * D);
-    if (nparts > cap) {
+    if (nparts > cap && own < 0) {
         // very many splits of one plane: per-element loop without staging
         for (int idx = tid; idx < G * D; idx += NT) {
             const int h = idx / D, c = idx % D;
@@ -551,8 +573,12 @@ __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c
     float* lss = scratch + cap * G;         // [part][G]: sums of exponentials
     float* Mh = scratch + 2 * cap * G;      // [G] maxima, [G] normalisers
     for (int i = tid; i < nparts * G; i += NT) {
-        wts[i] = __ldcg(pm + i);
-        lss[i] = __ldcg(pl + i);
+        if (i / G == own) {
+            own_state<D, G, W>(mg_m, mg_l, i % G, wts[i], lss[i]);
+        } else {
+            wts[i] = __ldcg(pm + i);
+            lss[i] = __ldcg(pl + i);
+        }
     }
     bool ok = sync();
     if (tid < G) {
@@ -580,9 +606,25 @@ __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c
         float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
         for (int s2 = 0; s2 < nparts; ++s2) {
+            if (s2 == own) continue;
             const float4 o = staged ? po[int64_t(s2) * (G * D / 4) + q4] : __ldcg(po + int64_t(s2) * (G * D / 4) + q4);
             const float f = wts[s2 * G + h];
             O.x += f * o.x; O.y += f * o.y; O.z += f * o.z; O.w += f * o.w;
+        }
+        if (own >= 0) {
+            // this CTA's part from the warps' stash, relative to its own maximum
+            float Mo, Lo;
+            own_state<D, G, W>(mg_m, mg_l, h, Mo, Lo);
+            if (Mo != NEG_INF_F) {
+                const float f = wts[own * G + h];
+                const int c = (q4 * 4) % D;
+#pragma unroll
+                for (int w2 = 0; w2 < W; ++w2) {
+                    const float fw = f * exp2f(mg_m[w2 * G + h] - Mo);
+                    const float4 o = *reinterpret_cast<const float4*>(mg_o + (w2 * G + h) * D + c);
+                    O.x += fw * o.x; O.y += fw * o.y; O.z += fw * o.z; O.w += fw * o.w;
+                }
+            }
         }
         const float Ls = Mh[G + h];
         const int c = (q4 * 4) % D;
@@ -612,11 +654,41 @@ template <typename T, int D, int G, int W, typename Sync>
 __device__ __forceinline__ bool flush_segment(const DecodeParams& p, const TileMeta& mt, int ctid, const SplitPlan& sp,
                                               const int* s_ts, float* mg_m, float* mg_l, float* mg_o, float* scratch,
                                               int scratch_floats, Sync& consumer_sync, int& s_last,
-                                              unsigned long long epoch, const MergeStage* stage = nullptr) {
+                                              unsigned long long epoch, const MergeStage* stage = nullptr,
+                                              int own_floats = 0, int snap_plane = -1,
+                                              unsigned long long snap = 0) {
     if (!consumer_sync()) return false;
     const int bg = mt.b * p.hkv + mt.g;
     const int slot = bg + int(blockIdx.x);
     const bool whole = mt.flags & kWhole;
+    // the fast merge below stages in the first own_floats of the scratch only (the rest holds
+    // the warps' stash, which it still reads)
+    const int own_cap = (own_floats - 2 * G) / (2 * G);
+    if (!whole && stage != nullptr && own_cap > 0) {
+        // The CTA's final segment: if every other part of the plane had arrived when ctid 0
+        // read the plane's counter a few tiles ago (snap, snap_plane: held by ctid 0 only, so
+        // every other condition here is uniform across the consumer threads), this CTA is the
+        // last one and merges straight from its warps' stash, without publishing its part (no
+        // fence and no arrival before the merge).
+        const int nt = ntiles_of(mt.len, mt.pad);
+        const int first = s_ts[mt.b] + mt.g * nt;
+        const int c0 = plan_cta_of(sp, first, bg), c1 = plan_cta_of(sp, first + nt - 1, bg);
+        if (c1 - c0 + 1 > own_cap) goto publish;
+        if (ctid == 0) {
+            const bool all_in = snap_plane == bg && (snap >> 20) == epoch &&
+                                unsigned(snap & 0xFFFFFull) + 1u == unsigned(c1 - c0 + 1);
+            if (all_in) fence_acq_rel_gpu();  // acquire what the relaxed read saw
+            s_last = all_in ? 2 : 0;
+        }
+        if (!consumer_sync()) return false;
+        if (s_last == 2) {
+            if (!merge_plane<T, D, G, W>(p, bg, c0, c1, int64_t(mt.b) * p.hq + mt.g * G, scratch, own_floats,
+                                         consumer_sync, ctid, stage, int(blockIdx.x) - c0, mg_m, mg_l, mg_o))
+                return false;
+            return consumer_sync();
+        }
+    }
+publish:
     for (int idx = ctid; idx < G * D; idx += W * 32) {
         const int h = idx / D, c = idx % D;
         float M = NEG_INF_F;
@@ -870,6 +942,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         return ok;
     };
 
+    int snap_plane = -1;
+    unsigned long long snap = 0;
     int it = 0;
     for (int t = start; t < end; ++t, ++it) {
         const int stage = it % STAGES;
@@ -883,6 +957,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         const TileMeta mt = meta[stage];
         const uint8_t* Kt = stage_mem + size_t(stage) * S::STAGE_BYTES;
         const uint8_t* Vt = Kt + S::KV_BYTES;
+        if (tid == 0 && t == max(start, end - 3)) {  // the final plane's counter, read ahead
+            snap_plane = mt.b * p.hkv + mt.g;
+            snap = ld_relaxed_gpu(p.ws_cnt + snap_plane);
+        }
         if (mt.flags & kFirst) cw.begin_segment(p, mt.b, mt.g);
         const int tok0 = mt.k * TILE + warp * TPW;  // first token of this warp's slice
         if (tok0 + TPW <= mt.len)
@@ -899,7 +977,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             const MergeStage ring{stage_mem, uint32_t(L::kStages), merge_bar};
             if (!flush_segment<T, D, G, W>(p, mt, tid, sp, s_ts, mg_m, mg_l, mg_o, p_s,
                                            int((L::kTileStart - L::kP) / sizeof(float)), consumer_sync, s_last,
-                                           epoch, t == end - 1 ? &ring : nullptr)) {
+                                           epoch, t == end - 1 ? &ring : nullptr,
+                                           int((L::kMergeM - L::kP) / sizeof(float)), snap_plane, snap)) {
                 record_status(YOCOPP_ETIMEOUT);
                 s_abort = 1;
                 break;

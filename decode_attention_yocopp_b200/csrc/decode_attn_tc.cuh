@@ -448,6 +448,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     };
 
     unsigned long long epoch = 0;  // epochs start at 1
+    int snap_plane = -1;
+    unsigned long long snap = 0;
     int it = 0;
     for (int t = start; t < end; ++t, ++it) {
         const int stage = it % STAGES;
@@ -460,6 +462,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             break;
         }
         const TileMeta mt = meta[stage];
+        if (ctid == 0 && t == max(start, end - 3)) {  // the final plane's counter, read ahead
+            snap_plane = mt.b * p.hkv + mt.g;
+            snap = ld_relaxed_gpu(p.ws_cnt + snap_plane);
+        }
         if (mt.flags & kFirst) cw.begin_segment();
         tc_fence_after();
         float sc[4];
@@ -496,7 +502,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             if (!flush_segment<__nv_bfloat16, S::D, G, W>(p, mt, ctid, sp, s_ts, mg_m, mg_l, mg_o, p_s,
                                                           int((L::kTileStart - L::kP) / sizeof(float)),
                                                           consumer_sync, s_last, epoch,
-                                                          t == end - 1 ? &ring : nullptr)) {
+                                                          t == end - 1 ? &ring : nullptr,
+                                                          int((L::kMergeM - L::kP) / sizeof(float)), snap_plane,
+                                                          snap)) {
                 record_status(YOCOPP_ETIMEOUT);
                 s_abort = 1;
                 break;

@@ -37,6 +37,11 @@
 // through separate two-slot rings, each refilled by its own producer lane as
 // soon as the last product reading the slot completes.
 //
+// prefill_tc_kernel<true> (yocopp_prefill_compose_attn) also composes the rows
+// it attends over, in the same launch: composition CTAs placed ahead of the
+// attention CTAs that read their rows, per-tile flags in the caller's
+// workspace (see the comment above the kernel).
+//
 // Warps: 0 = TMA producer (lane 0: Q and K, lane 1: V), 1 = MMA issuer and
 // tensor-memory owner, 2..5 = softmax and epilogue of head a, 6..9 = head b
 // (warp w reads TMEM lanes 32 (w mod 4) .. + 31).  Every wait is bounded; on
@@ -297,10 +302,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     int bidx = int(blockIdx.x);                                    // index in the attention order
     unsigned long long epoch = 0;
     if constexpr (FUSED) {
-        __shared__ unsigned long long s_ep;
-        if (tid == 0) s_ep = join_call(p.ws_gen, gridDim.x);
-        __syncthreads();
-        epoch = s_ep;
+        // every CTA reads the call's epoch (the last finished call's, + 1) and then arrives on
+        // the call counter, off the critical path: the composition CTAs in one of their
+        // composing threads, the attention CTAs in an idle lane of the loader warp
         const int per_attn = p.hkv * per_plane;
         int cb = -1, cjt = 0;
         if (bidx < p.q_tiles) {
@@ -317,13 +321,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             }
         }
         if (cb >= 0) {
+            __shared__ unsigned long long s_ep;
+            if (tid == 32) {
+                s_ep = __ldcg(p.ws_gen) + 1ull;
+                arrive_call(p.ws_gen, s_ep, gridDim.x);
+            }
             prefill_compose_tile(
                 p, cb, cjt, tid,
                 reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023)));
             fence_proxy_async_global();
             __threadfence();
             __syncthreads();
-            if (tid == 0) st_release_gpu(p.flags + int64_t(cb) * p.q_tiles + cjt, epoch);
+            if (tid == 0) st_release_gpu(p.flags + int64_t(cb) * p.q_tiles + cjt, s_ep);
             return;
         }
     }
@@ -344,15 +353,26 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         nq = p.n_uniform;
     }
     const int p0 = p.pos ? __ldg(p.pos + b) : 0;
+    // FUSED: a CTA with nothing to do still arrives on the call counter
+    auto leave = [&]() {
+        if constexpr (FUSED) {
+            if (tid == 0) arrive_call(p.ws_gen, __ldcg(p.ws_gen) + 1ull, gridDim.x);
+        }
+    };
     if (nq < 0) {
         if (tid == 0 && jt == 0 && g == 0 && rem % units == 0) record_status(YOCOPP_EDEVICE_CHECK);
+        leave();
         return;
     }
     if (p0 < 0 || int64_t(p0) + nq > p.capacity || nq > p.q_tiles * S::TQ) {
         if (tid == 0 && jt == 0 && g == 0 && rem % units == 0) record_status(YOCOPP_ECAPACITY);
+        leave();
         return;
     }
-    if (jt * S::TQ >= nq) return;
+    if (jt * S::TQ >= nq) {
+        leave();
+        return;
+    }
     const int kv_len = p0 + nq;
     const int jmax = min(jt * S::TQ + S::TQ - 1, nq - 1);
     const int ntk = (p0 + jmax) / S::TK + 1;        // key tiles 0 .. ntk-1 (causal)
@@ -401,6 +421,49 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 
     if (warp == 0) {
         // ------------------------------------------------------------------ producers
+        int composed_upto = -1;  // FUSED: query tiles of this call seen composed
+        if constexpr (FUSED) {
+            // the query tiles first (they are inputs, not composed rows)
+            if (lane == 0) {
+                prefetch_tensormap(&tmQ);
+                mbar_arrive_expect_tx(q_full, uint32_t((pair ? 2 : 1) * S::TILE_BYTES));
+                for (int x = 0; x < (pair ? 2 : 1); ++x)
+                    for (int bx = 0; bx < 2; ++bx)
+                        tma_load_3d(base + S::Q_OFF + x * S::TILE_BYTES + bx * S::BOXB, &tmQ, q_full, bx * 64,
+                                    h0 + x, qrow0 + jt * S::TQ);
+            }
+            if (lane == 2) epoch = __ldcg(p.ws_gen) + 1ull;
+            epoch = __shfl_sync(0xffffffffu, epoch, 2);
+            // one pass over every flag this CTA needs, 32 lanes x 4 loads in flight, then an
+            // acquire fence per lane and a warp barrier: the tiles found ready (normally all:
+            // their composition ran a sequence ahead) are not polled again
+            const int last_pos = min(ntk * S::TK, kv_len) - 1;
+            const int c_need = last_pos >= p0 ? (last_pos - p0) / S::TQ : -1;
+            const unsigned long long* fl = p.flags + int64_t(b) * p.q_tiles;
+            int first_missing = c_need + 1;
+            for (int c0 = 0; c0 <= c_need; c0 += 128) {
+                bool ready[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int c = c0 + 32 * k + lane;
+                    ready[k] = c > c_need || ld_relaxed_gpu(fl + c) == epoch;
+                }
+                unsigned miss = 0;
+#pragma unroll
+                for (int k = 0; k < 4 && miss == 0; ++k) {
+                    const unsigned m = __ballot_sync(0xffffffffu, !ready[k]);
+                    if (m) {
+                        miss = m;
+                        first_missing = c0 + 32 * k + __ffs(m) - 1;
+                    }
+                }
+                if (miss) break;
+            }
+            fence_acq_rel_gpu();
+            __syncwarp();
+            composed_upto = first_missing - 1;
+            if (lane == 2) arrive_call(p.ws_gen, epoch, gridDim.x);
+        }
         if (lane < 2) {
             const bool kl = lane == 0;   // lane 0: Q and the K ring; lane 1: the V ring
             const CUtensorMap* map = kl ? &tmK : &tmV;
@@ -410,7 +473,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             int issued = 0;
             bool ok = true;
             prefetch_tensormap(map);
-            if (kl) {
+            if (kl && !FUSED) {
                 prefetch_tensormap(&tmQ);
                 mbar_arrive_expect_tx(q_full, uint32_t((pair ? 2 : 1) * S::TILE_BYTES));
                 for (int x = 0; x < (pair ? 2 : 1); ++x)
@@ -420,7 +483,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             }
             const int plane_row = (b * p.hkv + g) * p.capacity;
             const int nsb = S::TK / p.boxr;  // boxes of boxr rows per tile (one per cache block)
-            int composed_upto = -1;          // FUSED: query tiles of this call seen composed
+            if constexpr (FUSED) fence_proxy_async_global();
             for (int t = 0; t < ntk; ++t) {
                 const int slot = t & 1;
                 if (s_abort || !mbar_wait(&empty[slot], ((t >> 1) & 1) ^ 1, p.wait_limit_ns)) {
@@ -432,13 +495,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     const int hi = min(t * S::TK + S::TK, kv_len) - 1;
                     if (hi >= p0) {
                         const int c_hi = (hi - p0) / S::TQ;
-                        while (ok && composed_upto < c_hi) {
-                            ok = wait_flag(p.flags + int64_t(b) * p.q_tiles + composed_upto + 1, epoch,
-                                           p.wait_limit_ns);
-                            if (ok) ++composed_upto;
+                        if (composed_upto < c_hi) {
+                            while (ok && composed_upto < c_hi) {
+                                ok = wait_flag(p.flags + int64_t(b) * p.q_tiles + composed_upto + 1, epoch,
+                                               p.wait_limit_ns);
+                                if (ok) ++composed_upto;
+                            }
+                            if (!ok) break;
+                            fence_proxy_async_global();
                         }
-                        if (!ok) break;
-                        fence_proxy_async_global();
                     }
                 }
                 if (kl && t == p.drop_k_tile && blockIdx.x == 0) continue;  // failure injection (tests)
