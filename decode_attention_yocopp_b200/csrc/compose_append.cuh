@@ -180,6 +180,10 @@ __global__ void __launch_bounds__(YOCOPP_COMPOSE_THREADS) compose_append_kernel(
     const int64_t stride = int64_t(gridDim.x) * blockDim.x;
     const ComposeCoef ck = make_coef(p.ak1, p.ak2, p.lam);
     const ComposeCoef cv = make_coef(p.av1, p.av2, p.lam);
+    // (token, head) rows fit 32 bits for every workload the host accepts below 2^31 rows: the
+    // row -> (token, head, sequence) arithmetic then runs in 32-bit integer division
+    const bool narrow = p.total_rows < (int64_t(1) << 31);
+    int bc = 0;  // ragged batches: this thread's last sequence (its chunks only move forward)
 
     for (int64_t i0 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i0 < nchunks; i0 += stride * U) {
         uint4 x1k[U], xik[U], x1v[U], xiv[U];
@@ -200,20 +204,42 @@ __global__ void __launch_bounds__(YOCOPP_COMPOSE_THREADS) compose_append_kernel(
             if (idx >= nchunks) continue;
             const int64_t row = idx / CPR;
             const int c = int(idx % CPR);
-            const int64_t tok = row / p.hkv;
-            const int h = int(row % p.hkv);
+            int64_t tok;
+            int h;
+            if (narrow) {
+                const uint32_t r32 = uint32_t(row), hk = uint32_t(p.hkv);
+                tok = int64_t(r32 / hk);
+                h = int(r32 - uint32_t(tok) * hk);
+            } else {
+                tok = row / p.hkv;
+                h = int(row % p.hkv);
+            }
             int b, j;
             if (p.cu_new == nullptr) {
-                b = int(tok / p.n_uniform);
+                if (narrow) {
+                    b = int(uint32_t(tok) / uint32_t(p.n_uniform));
+                } else {
+                    b = int(tok / p.n_uniform);
+                }
                 j = int(tok - int64_t(b) * p.n_uniform);
             } else {
-                // largest b with s_cu[b] <= tok (skips empty sequences)
-                int lo = 0, hi = p.batch;  // invariant: s_cu[lo] <= tok < s_cu[hi]
-                while (hi - lo > 1) {
-                    const int mid = (lo + hi) >> 1;
-                    if (s_cu[mid] <= tok) lo = mid; else hi = mid;
+                // largest b with s_cu[b] <= tok (skips empty sequences): a few steps on from this
+                // thread's last sequence, else a binary search
+                if (tok < s_cu[bc]) bc = 0;
+                int steps = 0;
+                while (bc + 1 < p.batch && s_cu[bc + 1] <= tok && steps < 4) {
+                    ++bc;
+                    ++steps;
                 }
-                b = lo;
+                if (bc + 1 < p.batch && s_cu[bc + 1] <= tok) {
+                    int lo = bc, hi = p.batch;  // invariant: s_cu[lo] <= tok < s_cu[hi]
+                    while (hi - lo > 1) {
+                        const int mid = (lo + hi) >> 1;
+                        if (s_cu[mid] <= tok) lo = mid; else hi = mid;
+                    }
+                    bc = lo;
+                }
+                b = bc;
                 j = int(tok - s_cu[b]);
             }
             const int64_t dst = cache_row_offset<ROWB>(p, b, j, h);
