@@ -31,7 +31,8 @@ EXPORTS = ("yocopp_compose_append", "yocopp_decode_attn_workspace_size", "yocopp
            "yocopp_get_device_status", "yocopp_status_string", "yocopp_version",
            "yocopp_testing_set_decode_fault", "yocopp_decode_attn_static", "yocopp_decode_attn_partial",
            "yocopp_decode_combine", "yocopp_decode_attn_fused", "yocopp_set_decode_kernel",
-           "yocopp_prefill_attn", "yocopp_prefill_compose_attn_workspace_size", "yocopp_prefill_compose_attn")
+           "yocopp_prefill_attn", "yocopp_prefill_compose_attn_workspace_size", "yocopp_prefill_compose_attn",
+           "yocopp_testing_set_decode_prefetch")
 
 
 class yocopp_cache(ctypes.Structure):
@@ -75,6 +76,8 @@ def load(path: Optional[str] = None):
     lib.yocopp_version.argtypes = []
     lib.yocopp_testing_set_decode_fault.restype = I32
     lib.yocopp_testing_set_decode_fault.argtypes = [I32, I64]
+    lib.yocopp_testing_set_decode_prefetch.restype = I32
+    lib.yocopp_testing_set_decode_prefetch.argtypes = [I32]
     lib.yocopp_decode_attn_partial.restype = I32
     lib.yocopp_decode_attn_partial.argtypes = [V, ctypes.POINTER(yocopp_cache), V, V, I32, ctypes.c_float, V, I64, V]
     lib.yocopp_set_decode_kernel.restype = I32
@@ -300,6 +303,10 @@ def yocopp_version() -> int:
 
 def yocopp_testing_set_decode_fault(drop_tile: int = -1, wait_limit_ns: int = 2_000_000_000) -> None:
     _check("yocopp_testing_set_decode_fault", load().yocopp_testing_set_decode_fault(int(drop_tile), int(wait_limit_ns)))
+
+
+def yocopp_testing_set_decode_prefetch(enabled: bool = True) -> None:
+    _check("yocopp_testing_set_decode_prefetch", load().yocopp_testing_set_decode_prefetch(int(enabled)))
 
 
 def alloc_workspace(cache: yocopp_cache, num_q_heads: int, device=None):

@@ -51,6 +51,7 @@ struct DecodeParams {
     int32_t num_ctas;
     int32_t seg_units;           // split plan: tiles' worth of work a segment's flush costs
     int32_t drop_tile;           // testing: a tile whose load is never issued (-1: none)
+    int32_t prefetch;            // 0: skip the L2 prefetch of the first tiles (testing)
     uint64_t wait_limit_ns;
     float* part_out;             // non-null: write unnormalised [batch][hq][D + 2] (o, m, l) instead of out
     float fa1k, fa2k, fa1v, fa2v;  // read-time composition (fused variant): lambda * alpha
@@ -117,10 +118,14 @@ __device__ __forceinline__ int clamp_len(const int32_t* lens, int b, int cap) {
     return len < 0 ? 0 : (len > cap ? cap : len);
 }
 
-// Block-wide exclusive prefix of tiles per sequence (x kv heads) into s_ts[0..batch].
+// Rendezvous of the first nthr threads of the block (nthr a multiple of 32).
+__device__ __forceinline__ void sync_first(int nthr) { asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory"); }
+
+// Exclusive prefix of tiles per sequence (x kv heads) into s_ts[0..batch], by the
+// block's first nthr threads.
 template <int TILE>
-__device__ void tile_prefix(const DecodeParams& p, int* s_ts, int* s_warp) {
-    const int nthr = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+__device__ void tile_prefix(const DecodeParams& p, int* s_ts, int* s_warp, int nthr) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int per = (p.batch + nthr - 1) / nthr;
     const int b0 = min(tid * per, p.batch), b1 = min(b0 + per, p.batch);
     int sum = 0;
@@ -136,7 +141,7 @@ __device__ void tile_prefix(const DecodeParams& p, int* s_ts, int* s_warp) {
         if (lane >= o) x += y;
     }
     if (lane == 31) s_warp[warp] = x;
-    __syncthreads();
+    sync_first(nthr);
     if (warp == 0) {
         int v = lane < (nthr >> 5) ? s_warp[lane] : 0;
 #pragma unroll
@@ -146,14 +151,14 @@ __device__ void tile_prefix(const DecodeParams& p, int* s_ts, int* s_warp) {
         }
         s_warp[lane] = v;
     }
-    __syncthreads();
+    sync_first(nthr);
     int excl = x - sum + (warp > 0 ? s_warp[warp - 1] : 0);
     for (int b = b0; b < b1; ++b) {
         s_ts[b] = excl;
         excl += ntiles_of(clamp_len(p.seq_lens, b, p.capacity), TILE) * p.hkv;
     }
     if (tid == nthr - 1) s_ts[p.batch] = excl;
-    __syncthreads();
+    sync_first(nthr);
 }
 
 // Split plan.  The tiles of all (sequence, kv-head) planes are flattened in
@@ -209,6 +214,85 @@ __device__ __forceinline__ int2 plan_range(const DecodeParams& p, const int* s_t
     int v = 0;
     if (lane < 2) v = plan_tile_at(p, s_ts, sp, int64_t(blockIdx.x + lane) * sp.unit);
     return make_int2(__shfl_sync(0xffffffffu, v, 0), __shfl_sync(0xffffffffu, v, 1));
+}
+
+// ---- the first tiles, prefetched before the previous kernel has finished ---
+// A kernel launched as a programmatic dependent may start while the previous
+// kernel still runs, and may read its inputs only after griddep_wait.  Until
+// then one warp guesses this CTA's plan from the lengths and block tables as
+// they stand (gpu-scope relaxed loads, which may be stale) and prefetches the
+// first tiles of its range into L2, so that the kernel's HBM reads start in
+// the previous kernel's tail.  The guess steers prefetches only: a stale length
+// or block costs a useless prefetch, never a wrong result, since everything the
+// kernel computes reads the inputs again after the wait.
+constexpr int kGuessMaxBatch = 256;  // larger batches skip the prefetch
+
+// The warp's guess of the prefix of tiles into s_g[0..batch], then L2 prefetches of
+// the first npf (<= 32) tiles of the guessed range.
+template <int TILE, int NBOX, int NSB_MAX>
+__device__ void prefetch_first_tiles(const DecodeParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                     int* s_g, int npf, int lane) {
+    constexpr int PER = kGuessMaxBatch / 32;
+    int n[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int b = i * 32 + lane;
+        const int raw = b < p.batch ? ld_relaxed_gpu(p.seq_lens + b) : 0;
+        n[i] = ntiles_of(raw < 0 ? 0 : min(raw, p.capacity), TILE) * p.hkv;
+    }
+    int base = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        if (i * 32 >= p.batch) break;
+        int x = n[i];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (i * 32 + lane < p.batch) s_g[i * 32 + lane] = base + x - n[i];
+        base += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) s_g[p.batch] = base;
+    __syncwarp();
+    const SplitPlan sp = make_plan(p, s_g, p.seg_units);
+    const int2 range = plan_range(p, s_g, sp, lane);
+    const int t = range.x + lane;
+    if (lane >= npf || t >= range.y) return;
+    int lo = 0, hi = p.batch;  // s_g[lo] <= t < s_g[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_g[mid] <= t) lo = mid; else hi = mid;
+    }
+    const int b = lo;
+    const int nt = (s_g[b + 1] - s_g[b]) / p.hkv;  // > 0: tile t lies in sequence b
+    const int local = t - s_g[b];
+    const int g = local / nt, k = local - g * nt;
+    if (p.block_table == nullptr) {
+        const int row = (b * p.hkv + g) * p.capacity + k * TILE;
+#pragma unroll
+        for (int bx = 0; bx < NBOX; ++bx) {
+            tma_prefetch_2d(tmK, bx * 64, row);
+            tma_prefetch_2d(tmV, bx * 64, row);
+        }
+        return;
+    }
+    const int raw = ld_relaxed_gpu(p.seq_lens + b);
+    const int len = raw < 0 ? 0 : min(raw, p.capacity);
+    const int nsb = TILE / p.boxr;
+#pragma unroll
+    for (int s = 0; s < NSB_MAX; ++s) {
+        const int tok = k * TILE + s * p.boxr;
+        if (s >= nsb || tok >= len) continue;
+        const int blk = ld_relaxed_gpu(p.block_table + int64_t(b) * p.mbps + tok / p.block_size);
+        if (blk < 0 || blk >= p.num_blocks) continue;
+        const int row = (blk * p.hkv + g) * p.block_size + tok % p.block_size;
+#pragma unroll
+        for (int bx = 0; bx < NBOX; ++bx) {
+            tma_prefetch_2d(tmK, bx * 64, row);
+            tma_prefetch_2d(tmV, bx * 64, row);
+        }
+    }
 }
 
 template <typename T, int D, int G, int W, int STAGES, bool FUSED = false>
@@ -781,7 +865,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     griddep_launch_dependents();
     __shared__ unsigned long long s_epoch;
     if (tid == 0) s_epoch = join_call(p.ws_gen, gridDim.x);
-    tile_prefix<TILE>(p, s_ts, s_warp);  // ends with __syncthreads()
+    tile_prefix<TILE>(p, s_ts, s_warp, blockDim.x);  // ends with a block-wide rendezvous
     const unsigned long long epoch = s_epoch;
     // sequences with no cached positions: zero output (CTA b mod grid writes it)
     for (int b = blockIdx.x; b < p.batch; b += p.num_ctas) {

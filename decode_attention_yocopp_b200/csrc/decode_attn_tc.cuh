@@ -12,7 +12,9 @@
 // alternate between tiles.
 //
 // Warps: 0 = TMA producer, 1 = MMA issuer and tensor-memory owner,
-// 2..5 = consumers.  A warp may only read the tensor-memory lanes of its
+// 2..5 = consumers, 6 = the L2 prefetch of the first tiles
+// (prefetch_first_tiles), which runs before the programmatic wait and exits;
+// the block-wide rendezvous of the others counts warps 0..5 only.  A warp may only read the tensor-memory lanes of its
 // quadrant (warp index mod 4), so consumer warp w owns tile rows
 // 32 (w mod 4) .. +31: one token per lane for the scores and the softmax,
 // then (as in the CUDA-core kernel) lanes own 16-byte channel chunks for the
@@ -38,13 +40,15 @@ struct TcShape {
     static constexpr int TMEM_COLS = 32;                         // two 16-column accumulators
     static constexpr uint32_t IDESC = umma_idesc_bf16(128, 16);
     static constexpr int NSB_MAX = 8;                            // sub-boxes per tile (block size 16)
+    static constexpr int WORKERS = (W + 2) * 32;                 // producer, MMA and consumer warps
+    static constexpr int THREADS = WORKERS + 32;                 // + the prefetch warp
 };
 static_assert(TcShape::STAGE_BYTES % 1024 == 0, "stage alignment");
 
 template <int G, int STAGES>
 struct TcSmem {
     using S = TcShape;
-    static constexpr size_t up16(size_t x) { return (x + 15) & ~size_t(15); }
+    __host__ __device__ static constexpr size_t up16(size_t x) { return (x + 15) & ~size_t(15); }
     static constexpr size_t kStages = size_t(STAGES) * S::STAGE_BYTES;
     static constexpr size_t kBars = kStages;  // full[S], empty[S], sfull[2], sempty[2], sync, merge
     static constexpr size_t kTmem = up16(kBars + (2 * STAGES + 6) * sizeof(uint64_t));
@@ -54,7 +58,11 @@ struct TcSmem {
     static constexpr size_t kMergeL = up16(kMergeM + size_t(S::W) * G * sizeof(float));
     static constexpr size_t kMergeO = up16(kMergeL + size_t(S::W) * G * sizeof(float));
     static constexpr size_t kTileStart = up16(kMergeO + size_t(S::W) * G * S::D * sizeof(float));
-    static size_t bytes(int batch) { return 1024 + kTileStart + size_t(batch + 1) * sizeof(int); }
+    // after s_ts, for the batches the prefetch warp handles: its guess of s_ts
+    __host__ __device__ static size_t guess_offset(int batch) { return up16(kTileStart + size_t(batch + 1) * sizeof(int)); }
+    static size_t bytes(int batch) {
+        return 1024 + guess_offset(batch) + (batch <= kGuessMaxBatch ? size_t(batch + 1) * sizeof(int) : 0);
+    }
 };
 
 // One consumer warp: 32 token rows of every tile.
@@ -185,8 +193,12 @@ struct TcConsumerWarp {
     }
 };
 
+#ifndef YOCOPP_DECODE_PREFETCH_TILES
+#define YOCOPP_DECODE_PREFETCH_TILES 2  // tiles per CTA prefetched into L2 before the programmatic wait
+#endif
+
 template <int G, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(TcShape::THREADS, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmQ, const DecodeParams p) {
     using S = TcShape;
@@ -236,6 +248,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         s_abort = 0;
         s_cdone = 0;
         s_epoch_ready = 0;
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        prefetch_tensormap(&tmQ);
+    }
+
+    if (warp == W + 2) {
+        // ---------------------------------------------- the prefetch, before the wait
+        if (YOCOPP_DECODE_PREFETCH_TILES > 0 && p.prefetch && p.batch <= kGuessMaxBatch)
+            prefetch_first_tiles<TILE, S::NBOX, S::NSB_MAX>(
+                p, &tmK, &tmV, reinterpret_cast<int*>(base + L::guess_offset(p.batch)), YOCOPP_DECODE_PREFETCH_TILES,
+                lane);
+        return;
     }
     // tensor memory needs no input: take it while the previous kernel may still run
     if (warp == 1) {
@@ -245,12 +269,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     tc_fence_before();
     griddep_wait();
     griddep_launch_dependents();
-    tile_prefix<TILE>(p, s_ts, s_warp);  // ends with __syncthreads()
+    tile_prefix<TILE>(p, s_ts, s_warp, S::WORKERS);  // ends with a rendezvous of warps 0..W+1
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     for (int b = blockIdx.x; b < p.batch; b += p.num_ctas) {
         if (s_ts[b + 1] != s_ts[b]) continue;
-        for (int idx = tid; idx < p.hq * S::D; idx += blockDim.x)
+        for (int idx = tid; idx < p.hq * S::D; idx += S::WORKERS)
             emit<__nv_bfloat16, S::D>(p, int64_t(b) * p.hq + idx / S::D, idx % S::D, NEG_INF_F, 0.f, 0.f);
     }
     const SplitPlan sp = make_plan(p, s_ts, p.seg_units);
@@ -264,12 +288,27 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 
     if (warp == 0) {
         // ------------------------------------------------------------------ producer
-        if (lane == 0) {
-            prefetch_tensormap(&tmK);
-            prefetch_tensormap(&tmV);
-            prefetch_tensormap(&tmQ);
-        }
+        // one tile's loads into a stage: K and V sub-boxes at rows r (-1: none), the group's q block
         const int nsb = TILE / p.boxr;
+        auto issue_tile = [&](int stage, const int* r, int b, int g, uint64_t* bar) {
+            uint32_t nvalid = 0;
+            for (int s = 0; s < nsb; ++s) nvalid += r[s] >= 0 ? 1u : 0u;
+            mbar_arrive_expect_tx(bar, nvalid * uint32_t(S::NBOX * p.boxr * 128 * 2) + uint32_t(S::Q_BYTES));
+            uint8_t* kdst = stage_mem + size_t(stage) * S::STAGE_BYTES;
+            uint8_t* vdst = kdst + S::KV_BYTES;
+            uint8_t* qdst = vdst + S::KV_BYTES;
+            for (int s = 0; s < nsb; ++s) {
+                if (r[s] < 0) continue;
+#pragma unroll
+                for (int bx = 0; bx < S::NBOX; ++bx) {
+                    const int off = bx * S::BOXB + s * p.boxr * 128;
+                    tma_load_2d(kdst + off, &tmK, bar, bx * 64, r[s]);
+                    tma_load_2d(vdst + off, &tmV, bar, bx * 64, r[s]);
+                }
+            }
+#pragma unroll
+            for (int bx = 0; bx < S::NBOX; ++bx) tma_load_2d(qdst + bx * S::QBOXB, &tmQ, bar, bx * 64, b * p.hq + g * G);
+        };
         int it = 0;
         int last_issued_it[STAGES];
 #pragma unroll
@@ -345,25 +384,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                 if (lane == 0) {
                     meta[stage] = m;
                     if (start + it != p.drop_tile) {
-                        uint32_t nvalid = 0;
-                        for (int s = 0; s < nsb; ++s) nvalid += r[s] >= 0 ? 1u : 0u;
-                        const uint32_t bytes = nvalid * uint32_t(S::NBOX * p.boxr * 128 * 2) + uint32_t(S::Q_BYTES);
-                        mbar_arrive_expect_tx(&full_bar[stage], bytes);
-                        uint8_t* kdst = stage_mem + size_t(stage) * S::STAGE_BYTES;
-                        uint8_t* vdst = kdst + S::KV_BYTES;
-                        uint8_t* qdst = vdst + S::KV_BYTES;
-                        for (int s = 0; s < nsb; ++s) {
-                            if (r[s] < 0) continue;
-#pragma unroll
-                            for (int bx = 0; bx < S::NBOX; ++bx) {
-                                const int off = bx * S::BOXB + s * p.boxr * 128;
-                                tma_load_2d(kdst + off, &tmK, &full_bar[stage], bx * 64, r[s]);
-                                tma_load_2d(vdst + off, &tmV, &full_bar[stage], bx * 64, r[s]);
-                            }
-                        }
-#pragma unroll
-                        for (int bx = 0; bx < S::NBOX; ++bx)
-                            tma_load_2d(qdst + bx * S::QBOXB, &tmQ, &full_bar[stage], bx * 64, m.b * p.hq + m.g * G);
+                        issue_tile(stage, r, m.b, m.g, &full_bar[stage]);
                         last_issued_it[stage] = it;
                     }
                 }

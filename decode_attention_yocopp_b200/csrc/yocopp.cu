@@ -25,6 +25,7 @@ constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
 // atomics, since launches may run on other host threads (relaxed: each value
 // stands alone).
 std::atomic<int> g_test_drop_tile{-1};
+std::atomic<int> g_test_prefetch{1};
 std::atomic<int> g_decode_kernel{0};  // 0 / 2: tensor-core scores where supported, 1: CUDA-core scores
 std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
 
@@ -209,7 +210,7 @@ int32_t launch_decode_tc(const CUtensorMap& tk, const CUtensorMap& tv, const CUt
     if (smem > max_dyn[dev]) return YOCOPP_EINVAL;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(unsigned(p.num_ctas), 1, 1);
-    lc.blockDim = dim3(192, 1, 1);
+    lc.blockDim = dim3(TcShape::THREADS, 1, 1);
     lc.dynamicSmemBytes = smem;
     lc.stream = st;
     cudaLaunchAttribute attr[1];
@@ -383,6 +384,12 @@ int32_t yocopp_testing_set_decode_fault(int32_t drop_tile, int64_t wait_limit_ns
     return YOCOPP_OK;
 }
 
+int32_t yocopp_testing_set_decode_prefetch(int32_t enabled) {
+    if (enabled != 0 && enabled != 1) return YOCOPP_EINVAL;
+    g_test_prefetch.store(enabled, std::memory_order_relaxed);
+    return YOCOPP_OK;
+}
+
 int32_t yocopp_compose_append(const void* K1, const void* V1, const void* Ki, const void* Vi,
                               const float alpha[4], float lambda, const yocopp_cache* cache,
                               const int32_t* pos, const int32_t* cu_new, int32_t n_uniform,
@@ -530,6 +537,7 @@ static int32_t decode_attn_impl(const void* q, const yocopp_cache* cache, const 
     p.num_ctas = num_ctas;
     p.seg_units = YOCOPP_DECODE_SEG_UNITS;
     p.drop_tile = g_test_drop_tile.load(std::memory_order_relaxed);
+    p.prefetch = g_test_prefetch.load(std::memory_order_relaxed);
     p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
     p.part_out = part_out;
     p.fa1k = fused ? fused->coef[0] : 0.f;

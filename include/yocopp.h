@@ -379,6 +379,19 @@ int32_t yocopp_set_decode_kernel(int32_t which);
  */
 int32_t yocopp_testing_set_decode_fault(int32_t drop_tile, int64_t wait_limit_ns);
 
+/*
+ * yocopp_testing_set_decode_prefetch - switch for the early L2 prefetch of the
+ * tensor-core decode kernel (on by default).  Host-side, process-wide; affects
+ * later decode launches.  Launched while the previous kernel in the stream
+ * still runs, that kernel guesses, before its programmatic wait, each CTA's
+ * first tiles from the lengths and block tables as they stand and prefetches
+ * them into L2; everything it computes reads the inputs again after the wait.
+ *   enabled : 1 = prefetch (default), 0 = no prefetch.
+ * The results are the same bits either way.  Returns YOCOPP_EINVAL for other
+ * values.
+ */
+int32_t yocopp_testing_set_decode_prefetch(int32_t enabled);
+
 #ifdef __cplusplus
 }
 #endif
