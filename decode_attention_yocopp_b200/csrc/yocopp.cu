@@ -431,6 +431,13 @@ int32_t yocopp_compose_append(const void* K1, const void* V1, const void* Ki, co
     p.block_size = cache->block_table ? cache->block_size : 0;
     p.mbps = cache->block_table ? cache->max_blocks_per_seq : 0;
     p.num_blocks = cache->block_table ? cache->num_blocks : 0;
+    const FastDiv dh = make_fast_div(uint32_t(cache->num_kv_heads)), dn = make_fast_div(uint32_t(n_uniform > 0 ? n_uniform : 1));
+    p.hkv_m = dh.m;
+    p.hkv_s = dh.s;
+    p.nu_m = dn.m;
+    p.nu_s = dn.s;
+    p.bs_log2 = 0;
+    while (cache->block_table && (1 << p.bs_log2) < cache->block_size) ++p.bs_log2;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int rowb = cache->head_dim * elem_bytes(cache->dtype);
     if (cache->dtype == YOCOPP_BF16)

@@ -119,6 +119,17 @@ def test_paged_small_blocks(y, orc):
     _run(y, orc, dtype="bf16", d=128, hkv=4, n_per_seq=[37, 5, 90], pos=[0, 16, 7], paged=True, block_size=16)
 
 
+def test_odd_divisors_uniform(y, orc):
+    # 3 KV heads and 7 new rows per sequence: the kernel's row -> (token, head, sequence)
+    # divisions by multiply-high with divisors that are not powers of two
+    _run(y, orc, dtype="bf16", d=128, hkv=3, n_per_seq=[7] * 5, pos=[0, 1, 9, 30, 2], paged=False, capacity=40)
+
+
+def test_odd_divisors_ragged_paged(y, orc):
+    _run(y, orc, dtype="bf16", d=128, hkv=3, n_per_seq=[0, 77, 5, 130, 1], pos=[0, 0, 31, 2, 64], paged=True,
+         block_size=32)
+
+
 def test_head_dim_64_bf16(y, orc):
     _run(y, orc, dtype="bf16", d=64, hkv=2, n_per_seq=[130, 3], pos=[0, 9], paged=False)
 

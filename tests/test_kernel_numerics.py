@@ -140,14 +140,15 @@ def test_monotone_across_integer_boundaries():
 # ---------------------------------------------------------------------------
 # The composition kernel's rounding (the stored
 # value is the exact composition rounded once).  Its fast path forms
-# lambda * (a1 * x1 + a2 * xi) in fp32 with error-free transformations
-# (TwoProduct by FMA, Knuth's TwoSum) and rounds the fp32 result y to bf16;
-# a y whose low 16 bits lie within 2 fp32 ulps of a bf16 rounding midpoint is
-# sent to an fp64 path that reproduces the oracle's evaluation.  The claim to
-# pin: wherever the detector lets y through, rounding y gives the same bf16 as
-# rounding the oracle's value once.  The replay below follows the kernel's
-# fp32 steps; every fused multiply-add is reproduced exactly (an fp64 product
-# that is exact, an fp64 TwoSum, and a tie decided by the TwoSum's error).
+# lambda * (a1 * x1 + a2 * xi) in fp32 from exact product errors (TwoProduct
+# by FMA), y = fl(lambda s - fl(lambda fl(n1 + n2))) with s = fl(p1 + p2), and
+# rounds y to bf16; a y whose low 16 bits lie within 3 fp32 ulps of a bf16
+# rounding midpoint is sent to an fp64 path that reproduces the oracle's
+# evaluation.  The claim to pin: wherever the detector lets y through,
+# rounding y gives the same bf16 as rounding the oracle's value once.  The
+# replay below follows the kernel's fp32 steps; every fused multiply-add is
+# reproduced exactly (an fp64 product that is exact, an fp64 TwoSum, and a tie
+# decided by the TwoSum's error).
 
 LAM = 35.0
 
@@ -162,10 +163,7 @@ def kernel_compose_fast(x1, xi, a1, a2, lam):
     p2 = (a2 * xi).astype(f)
     n2 = _fma32(-a2, xi, p2)
     s = (p1 + p2).astype(f)
-    bb = (s - p1).astype(f)
-    err = ((p1 - (s - bb).astype(f)).astype(f) + (p2 - bb).astype(f)).astype(f)
-    lo = (err - (n1 + n2).astype(f)).astype(f)
-    return _fma32(lam, s, (lam * lo).astype(f))
+    return _fma32(lam, s, (-lam * (n1 + n2).astype(f)).astype(f))
 
 
 COMPOSE_SRC = os.path.join(ROOT, "decode_attention_yocopp_b200", "csrc", "compose_append.cuh")
@@ -174,14 +172,14 @@ COMPOSE_SRC = os.path.join(ROOT, "decode_attention_yocopp_b200", "csrc", "compos
 def test_replay_matches_kernel_source():
     # the detector and the fast path's steps replayed here are the kernel's
     src = open(COMPOSE_SRC).read()
-    assert "((__float_as_uint(y) - 0x7FFEu) & 0xFFFFu) <= 4u" in src
-    for step in ("fmul2(a1, x1)", "ffma2(na1, x1, p1)", "fadd2(p1, p2)", "fsub2(s, p1)",
-                 "fsub2(err, fadd2(n1, n2))", "ffma2(lam, s, fmul2(lam, lo))"):
+    assert "((__float_as_uint(y) - 0x7FFDu) & 0xFFFFu) <= 6u" in src
+    for step in ("fmul2(a1, x1)", "ffma2(na1, x1, p1)", "fmul2(a2, xi)", "ffma2(na2, xi, p2)", "fadd2(p1, p2)",
+                 "ffma2(lam, s, fmul2(nlam, fadd2(n1, n2)))", "c.nlam = make_float2(-lam, -lam)"):
         assert step in src, step
 
 
 def _near_midpoint(y):
-    return ((y.view(np.uint32) - np.uint32(0x7FFE)) & np.uint32(0xFFFF)) <= 4
+    return ((y.view(np.uint32) - np.uint32(0x7FFD)) & np.uint32(0xFFFF)) <= 6
 
 
 def _rne_bf16(y):
@@ -207,8 +205,10 @@ def _check_compose_rounding(orc, x1_bits, xi_bits, a1, a2):
     fast = ~_near_midpoint(y)
     bad = fast & (_rne_bf16(y) != want)
     assert not bad.any(), (int(bad.sum()), exact[bad][:4], y[bad][:4])
-    # the fp32 result is within two fp32 ulps of the oracle's value
-    assert np.all(np.abs(y.astype(np.float64) - exact) <= 2 * np.spacing(np.abs(y)).astype(np.float64) + 1e-300)
+    # the fp32 result is within two fp32 ulps of the oracle's value (the bound the detector's
+    # window of 3 ulps relies on, with one ulp to spare for the second-order terms)
+    err = np.abs(y.astype(np.float64) - exact)
+    assert np.all(err <= 2 * np.spacing(np.abs(y)).astype(np.float64) * (1 + 2.0 ** -20) + 1e-300)
     return float(1.0 - fast.mean())
 
 
@@ -225,7 +225,7 @@ def test_compose_fast_path_rounds_once_on_workload_weights(orc, seed):
     a1 = rng.uniform(-0.05, 0.05)
     a2 = 1 / 35 + rng.uniform(-0.05, 0.05)
     slow = _check_compose_rounding(orc, x1, xi, a1, a2)
-    assert slow < 2e-4   # the fp64 path stays rare (about 5 in 2^16)
+    assert slow < 2.5e-4   # the fp64 path stays rare (about 7 in 2^16)
 
 
 def test_compose_fast_path_under_cancellation(orc):
