@@ -587,15 +587,15 @@ def run_leg(cfg, args, rank, world, local):
         "decode_attention": {"kernel": dk, "kv_read_gbs_job": round(kv_all / (t_attn_max * 1e-3) / 1e9, 1),
                              "achieved_gbs_per_layer": round(ach_attn, 1),
                              "ms_per_layer": round(sum(per_layer) / len(per_layer), 4),
-                             "frac_of_measured": round(ach_attn / peak, 4),
+                             "frac": round(ach_attn / peak, 4),
                              "frac_of_nominal": round(ach_attn / NOMINAL_HBM_GBS, 4), "peak": peak,
                              "peak_kind": peak_kind, "traffic": ncu_traffic(dk, w.name),
                              "algorithmic_bytes_per_launch": w.kv_bytes()},
         "compose": {"kernel": "compose_append_kernel (prefill size)",
                     "gbs_job": round(comp_all / (t_prefill_max * 1e-3) / 1e9, 1),
                     "achieved_gbs_per_launch": round(ach_comp, 1),
-                    "frac_of_measured": round(ach_comp / peak, 4),
-                    "frac_of_nominal": round(ach_comp / NOMINAL_HBM_GBS, 4),
+                    "frac": round(ach_comp / peak, 4),
+                    "frac_of_nominal": round(ach_comp / NOMINAL_HBM_GBS, 4), "peak": peak, "peak_kind": peak_kind,
                     "traffic": ncu_traffic("compose_append_kernel", w.name),
                     "algorithmic_bytes_per_launch": w.compose_bytes(w.total_prefill)},
         "decode_tok_s": round(tok_all / (t_decode_max * 1e-3), 1),
