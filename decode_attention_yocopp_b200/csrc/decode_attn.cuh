@@ -599,8 +599,10 @@ struct MergeStage {
 // (slots plane + cta) and write the group's outputs.  Run by the W consumer
 // warps of the last CTA to arrive.  One parallel pass stages every part's
 // maximum and sum in shared memory (the probability and warp-merge areas,
-// free at this point); weights e^{m_s - M} are formed once per (part, head);
-// then each thread accumulates 4 channels.  With a staging area large enough,
+// free at this point); after one rendezvous, the lanes that hold a head's
+// channels form its maximum, the weights 2^(m_s - M) (once per part and head)
+// and the normaliser among themselves, and each thread accumulates its 4
+// channels.  With a staging area large enough,
 // the parts' value sums (contiguous slots) come in with one bulk copy issued
 // first, so that the whole merge costs one round trip to L2 for them instead
 // of one per few parts.
@@ -626,7 +628,7 @@ __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c
                                             const float* mg_l = nullptr, const float* mg_o = nullptr) {
     constexpr int NT = W * 32;
     const int nparts = c1 - c0 + 1;
-    const int cap = (scratch_floats - 2 * G) / (2 * G);  // parts that fit the staging area
+    const int cap = scratch_floats / (2 * G);  // parts whose maxima and sums fit the scratch
     const float* pm = p.ws_m + int64_t(bg + c0) * G;
     const float* pl = p.ws_l + int64_t(bg + c0) * G;
     const float4* po = reinterpret_cast<const float4*>(p.ws_o + int64_t(bg + c0) * G * D);
@@ -655,7 +657,6 @@ __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c
     }
     float* wts = scratch;                   // [part][G]: maxima, then weights
     float* lss = scratch + cap * G;         // [part][G]: sums of exponentials
-    float* Mh = scratch + 2 * cap * G;      // [G] maxima, [G] normalisers
     for (int i = tid; i < nparts * G; i += NT) {
         if (i / G == own) {
             own_state<D, G, W>(mg_m, mg_l, i % G, wts[i], lss[i]);
@@ -665,28 +666,38 @@ __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c
         }
     }
     bool ok = sync();
-    if (tid < G) {
-        float M = NEG_INF_F;
-        for (int s2 = 0; s2 < nparts; ++s2) M = fmaxf(M, wts[s2 * G + tid]);
-        Mh[tid] = M;
-    }
-    ok = sync() && ok;
-    for (int i = tid; i < nparts * G; i += NT) wts[i] = exp2f(wts[i] - Mh[i % G]);
-    ok = sync() && ok;
-    if (tid < G) {
-        float Ls = 0.f;
-        for (int s2 = 0; s2 < nparts; ++s2) Ls += wts[s2 * G + tid] * lss[s2 * G + tid];
-        Mh[G + tid] = Ls;
-    }
-    ok = sync() && ok;
     if (staged) {
         // every thread waits (bounded) for the bulk copy; a warp continues only if all its lanes saw it
         ok = __all_sync(0xffffffffu, mbar_wait(stage->bar, 0, p.wait_limit_ns)) && ok;
         if (!ok) return false;
         po = reinterpret_cast<const float4*>(stage->buf);
     }
-    for (int q4 = tid; q4 < G * D / 4; q4 += NT) {
-        const int h = (q4 * 4) / D;
+    // A thread holds 4 channels, so a head's D channels are LPH = D / 4 lanes of one warp; those
+    // lanes form the head's maximum, weights 2^(m_s - M) (in place of the maxima, read back by
+    // the same lanes) and normaliser among themselves, with shuffles and no rendezvous.
+    constexpr int LPH = D / 4;
+    static_assert(32 % LPH == 0, "a head's lanes within one warp");
+    const int lane = tid & 31, g = lane % LPH;
+    for (int q0 = tid - lane; q0 < G * D / 4; q0 += NT) {  // warp-uniform trip count
+        const int q4 = q0 + lane;
+        const bool act = q4 < G * D / 4;
+        const int h = act ? (q4 * 4) / D : 0;
+        float M = NEG_INF_F;
+        if (act)
+            for (int s2 = g; s2 < nparts; s2 += LPH) M = fmaxf(M, wts[s2 * G + h]);
+#pragma unroll
+        for (int o = LPH / 2; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o, LPH));
+        float Ls = 0.f;
+        if (act)
+            for (int s2 = g; s2 < nparts; s2 += LPH) {
+                const float f = M != NEG_INF_F ? exp2f(wts[s2 * G + h] - M) : 0.f;
+                wts[s2 * G + h] = f;
+                Ls += f * lss[s2 * G + h];
+            }
+#pragma unroll
+        for (int o = LPH / 2; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o, LPH);
+        __syncwarp();
+        if (!act) continue;
         float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
         for (int s2 = 0; s2 < nparts; ++s2) {
@@ -710,13 +721,12 @@ __device__ __forceinline__ bool merge_plane(const DecodeParams& p, int bg, int c
                 }
             }
         }
-        const float Ls = Mh[G + h];
         const int c = (q4 * 4) % D;
         if (p.part_out != nullptr) {
-            emit<T, D>(p, out_row0 + h, c + 0, Mh[h], Ls, O.x);
-            emit<T, D>(p, out_row0 + h, c + 1, Mh[h], Ls, O.y);
-            emit<T, D>(p, out_row0 + h, c + 2, Mh[h], Ls, O.z);
-            emit<T, D>(p, out_row0 + h, c + 3, Mh[h], Ls, O.w);
+            emit<T, D>(p, out_row0 + h, c + 0, M, Ls, O.x);
+            emit<T, D>(p, out_row0 + h, c + 1, M, Ls, O.y);
+            emit<T, D>(p, out_row0 + h, c + 2, M, Ls, O.z);
+            emit<T, D>(p, out_row0 + h, c + 3, M, Ls, O.w);
         } else {
             const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
             const int64_t o0 = out_row0 * D + int64_t(q4) * 4;
