@@ -130,6 +130,13 @@ def test_odd_divisors_ragged_paged(y, orc):
          block_size=32)
 
 
+@pytest.mark.parametrize("bs", [128, 256])
+def test_paged_large_blocks(y, orc, bs):
+    # block sizes above a 128-row tile: the block shift and mask of the kernel's row arithmetic
+    _run(y, orc, dtype="bf16", d=128, hkv=2, n_per_seq=[300, 1, bs + 5], pos=[0, bs - 1, 7], paged=True,
+         block_size=bs)
+
+
 def test_head_dim_64_bf16(y, orc):
     _run(y, orc, dtype="bf16", d=64, hkv=2, n_per_seq=[130, 3], pos=[0, 9], paged=False)
 

@@ -67,10 +67,16 @@ CASES = [
     dict(seed=34, lens=[1, 129], hkv=2, G=1),
     # more sequences than the guess handles: no prefetch
     dict(seed=35, lens=[40 + (7 * b) % 200 for b in range(300)], hkv=1, G=4),
+    # the largest batch the guess handles, and one more
+    dict(seed=37, lens=[1 + (13 * b) % 300 for b in range(256)], hkv=1, G=2),
+    dict(seed=38, lens=[1 + (13 * b) % 300 for b in range(257)], hkv=1, G=2),
+    # paged with blocks of 256 rows (two 128-row boxes per block)
+    dict(seed=39, lens=[700, 256, 1], hkv=2, G=4, paged=True, block_size=256),
 ]
 
 
-@pytest.mark.parametrize("spec", CASES, ids=["b1_long", "ragged_paged16", "paged64_g2", "tiny", "batch300"])
+@pytest.mark.parametrize("spec", CASES, ids=["b1_long", "ragged_paged16", "paged64_g2", "tiny", "batch300",
+                                              "batch256", "batch257", "paged256"])
 def test_prefetch_same_bits_and_oracle(y, orc, spec):
     case = DecodeCase(key_scale=2.0, **spec)
     on = _run(y, case, True, repeats=3)
