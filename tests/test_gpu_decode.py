@@ -132,6 +132,13 @@ def test_paged_block32_group1(y, orc):
     run_case(y, orc, dtype="bf16", d=128, hkv=4, G=1, lens=[500, 31, 1200], paged=True, block_size=32)
 
 
+@pytest.mark.parametrize("G", [1, 2])
+def test_long_context_small_groups(y, orc, G):
+    # one long sequence per call: every (sequence, kv-head) plane is split over many CTAs and
+    # merged with 1 or 2 query heads per kv head
+    run_case(y, orc, dtype="bf16", d=128, hkv=8, G=G, lens=[12000], key_scale=2.0)
+
+
 def test_head_dim_64_bf16(y, orc):
     run_case(y, orc, dtype="bf16", d=64, hkv=4, G=4, lens=[1, 100, 2049, 64])
 
