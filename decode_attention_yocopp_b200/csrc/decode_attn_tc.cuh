@@ -14,12 +14,12 @@
 // Warps: 0 = TMA producer, 1 = MMA issuer and tensor-memory owner,
 // 2..5 = consumers, 6 = the L2 prefetch of the first tiles
 // (prefetch_first_tiles), which runs before the programmatic wait and exits;
-// the block-wide rendezvous of the others counts warps 0..5 only.  A warp may only read the tensor-memory lanes of its
-// quadrant (warp index mod 4), so consumer warp w owns tile rows
-// 32 (w mod 4) .. +31: one token per lane for the scores and the softmax,
-// then (as in the CUDA-core kernel) lanes own 16-byte channel chunks for the
-// value sum.  Every wait is bounded; the tensor memory is freed on every exit
-// path after the MMAs in flight have completed.
+// the block-wide rendezvous of the others counts warps 0..5 only.  A warp may
+// only read the tensor-memory lanes of its quadrant (warp index mod 4), so
+// consumer warp w owns tile rows 32 (w mod 4) .. +31: one token per lane for
+// the scores and the softmax, then (as in the CUDA-core kernel) lanes own
+// 16-byte channel chunks for the value sum.  Every wait is bounded; the tensor
+// memory is freed on every exit path after the MMAs in flight have completed.
 #pragma once
 
 #include "decode_attn.cuh"
